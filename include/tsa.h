@@ -1,0 +1,180 @@
+/*
+ * tsa.h: C ABI of libtsa, the Token Sparse Attention layer for NVIDIA B200 (sm_100a).
+ *
+ * The method is from "Token Sparse Attention: Efficient Long-Context Inference with
+ * Interleaved Token Selection".  Page citations below:
+ *   [notes] the papernotes.org notes on that paper (方法详解 › 整体框架; 关键设计 1
+ *           Compress-then-Decompress; 关键设计 2 Dynamic Token Coverage);
+ *   [blog]  the bxzpzcl.cn post (§1.1 核心算法实现细节; §2.1 重要性评估机制);
+ *   [gist]  the gist.science summary (§2 Methodology: Core Architecture; Dynamic
+ *           Token Coverage).
+ *
+ * Conventions shared by every call
+ *   Memory   The caller owns every buffer.  All pointers are device pointers on the
+ *            current CUDA device, 16-byte aligned and densely packed in the layout
+ *            stated.  The library allocates, frees and synchronises nothing
+ *            (tsa_get_device_status is the one call that synchronises).
+ *   Streams  Every call only enqueues work on `stream` (a cudaStream_t passed as
+ *            void*, NULL = legacy default stream) and returns.  L' stays on the
+ *            device, so no call reads results back to the host.
+ *   Layouts  Q  [B, L, H, d];  K, V [B, L, Hkv, d];  X, Y [B, L, H*d]  (row-major);
+ *            s_h [B, H, L] fp32;  s_l [B, L] fp32;  Lkeep [B] int32;
+ *            idx [B, H, L] int32;  Qh, Kh, Vh, Oh [B, H, L, d] (compressed, head-major).
+ *            Query head h reads KV head h / (H / Hkv).
+ *   Types    dtype TSA_BF16: Q, K, V, X, Y, Qh, Kh, Vh, Oh are bfloat16, with fp32
+ *            accumulation everywhere.  dtype TSA_F32: the same tensors are fp32.
+ *            d must be 64 or 128.  G * min(q, L) <= 256 where G = H / Hkv.
+ *   Errors   Each call returns a status and never aborts.  Argument errors are found
+ *            on the host before anything is enqueued.  A failed launch returns
+ *            TSA_ERR_CUDA.  tsa_last_error() gives a message for the calling thread.
+ *            Errors found on the device (a bounded wait that ran out, a score that is
+ *            not a finite value in [0, 1]) are recorded in the workspace's error word
+ *            and returned by tsa_get_device_status.
+ *   Workspace `ws` is caller-owned device scratch of at least tsa_workspace_size()
+ *            bytes (tsa_layer_workspace_size() for tsa_layer), 256-byte aligned,
+ *            zero-filled once before its first use.  Calls that share a workspace
+ *            must be ordered on one stream.
+ */
+#ifndef TSA_H_
+#define TSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TSA_API __attribute__((visibility("default")))
+#else
+#define TSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TSA_OK = 0,
+    TSA_ERR_INVALID_ARG = 1,    /* a null pointer, a bad size, tau or scale      */
+    TSA_ERR_ALIGNMENT = 2,      /* a pointer that is not 16-byte aligned          */
+    TSA_ERR_UNSUPPORTED = 3,    /* a shape or dtype this build does not implement */
+    TSA_ERR_WORKSPACE = 4,      /* workspace too small or misaligned              */
+    TSA_ERR_CUDA = 5,           /* a CUDA runtime or launch error                 */
+    TSA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait ran out             */
+    TSA_ERR_NONFINITE = 7       /* a score outside [0, 1] or not finite           */
+} tsa_status;
+
+typedef enum { TSA_F32 = 0, TSA_BF16 = 1 } tsa_dtype;
+
+typedef struct {
+    int32_t B;     /* batch                                   */
+    int32_t L;     /* tokens per sequence, 1 <= L <= 2^21      */
+    int32_t H;     /* query heads                              */
+    int32_t Hkv;   /* key/value heads, H % Hkv == 0            */
+    int32_t d;     /* head dimension, 64 or 128                */
+    int32_t dtype; /* tsa_dtype                                */
+} tsa_dims;
+
+/* Bytes of workspace needed by tsa_score, tsa_budget, tsa_select and tsa_attn for
+ * these dims and q (0 on invalid arguments). */
+TSA_API size_t tsa_workspace_size(const tsa_dims *dims, int32_t q);
+
+/* Bytes of workspace needed by tsa_layer: the above plus room for every
+ * intermediate (s_h, s_l, Lkeep, idx, Qh, Kh, Vh, Oh). */
+TSA_API size_t tsa_layer_workspace_size(const tsa_dims *dims, int32_t q);
+
+/* Dynamic Token Coverage scoring ([notes] 关键设计 2; [blog] §2.1; [gist] §2).
+ * For each batch b, query head h and each of the last q_eff = min(q, L) positions
+ * p = L - q_eff + i, the softmax over keys t <= p of scale * <Q[b,p,h], K[b,t,kv(h)]>
+ * gives A[i, t]; s_h[b,h,t] = sum_i A[i,t].  Then u[t] = sum_h s_h[b,h,t] and
+ * s_l[b,t] = u[t] / sum_t u[t].  Causal scoring and the shared scale are readings of
+ * the pages.  Deterministic: every sum runs in a fixed order.
+ * Q [B,L,H,d], K [B,L,Hkv,d]; s_h [B,H,L] and s_l [B,L] fp32 outputs.  scale > 0
+ * (normally 1/sqrt(d)). */
+TSA_API tsa_status tsa_score(const tsa_dims *dims, const void *Q, const void *K, int32_t q,
+                     float scale, float *s_h, float *s_l, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/* Coverage budget ([notes] 关键设计 2; [blog] §2.1 层级预算分配; [gist] §2 Budget
+ * Allocation).  Sort s_l[b,:] ascending and find the smallest k whose cumulative mass
+ * reaches tau; Lkeep[b] = L - k (k = L, so Lkeep = 0, if it is never reached).  The
+ * cumulative mass is exact: each s_l is taken as floor(s_l * 2^62) in uint64 and
+ * compared with ceil(tau * 2^62).  s_l values must lie in [0, 1] and sum to at most 4
+ * (tsa_score's sum to 1).  0 <= tau < 1.  Lkeep [B] int32 device output. */
+TSA_API tsa_status tsa_budget(const tsa_dims *dims, const float *s_l, double tau, int32_t *Lkeep,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/* Per-head top-L' selection ([notes] 关键设计 2; [gist] §2 Head-Wise Selection).
+ * For each (b, h): the Lkeep[b] tokens with the largest s_h[b,h,:], ties to the lower
+ * token index, written to idx[b,h,0:Lkeep[b]] in ascending token order; the other
+ * L - Lkeep[b] tokens follow in idx[b,h,Lkeep[b]:L], also ascending, so each row of
+ * idx is a permutation of 0..L-1.  Lkeep is read on the device. */
+TSA_API tsa_status tsa_select(const tsa_dims *dims, const float *s_h, const int32_t *Lkeep,
+                      int32_t *idx, void *ws, size_t ws_bytes, void *stream);
+
+/* Compress ([notes] 整体框架, 关键设计 1; [blog] §1.1 压缩阶段; [gist] §2 Compression).
+ * For i < Lkeep[b]: Qh[b,h,i] = Q[b,idx[b,h,i],h], Kh[b,h,i] = K[b,idx[b,h,i],kv(h)],
+ * Vh likewise.  Rows i in [Lkeep[b], min(L, ceil128(Lkeep[b]))) of Qh, Kh, Vh are
+ * zero-filled (the attention kernel reads whole 128-row tiles); later rows are not
+ * written. */
+TSA_API tsa_status tsa_gather_qkv(const tsa_dims *dims, const void *Q, const void *K,
+                          const void *V, const int32_t *idx, const int32_t *Lkeep,
+                          void *Qh, void *Kh, void *Vh, void *stream);
+
+/* Attention ([notes] 整体框架; [blog] §1.1 softmax(Q̂K̂ᵀ/√d)V̂).
+ * dense == 0 (compressed): for each (b, h) and i < Lkeep[b],
+ *   Oh[b,h,i] = sum_{j<=i} softmax_j(scale * <Qh[b,h,i], Kh[b,h,j]>) Vh[b,h,j];
+ *   inputs and output are [B,H,L,d].  Because idx lists kept tokens in ascending
+ *   order, j <= i is the causal mask on original positions.  Rows of Kh/Vh in
+ *   [Lkeep[b], ceil128(Lkeep[b])) must hold finite values (tsa_gather_qkv zeroes
+ *   them).  Rows i >= Lkeep[b] of Oh are not written.
+ * dense == 1: dense causal GQA attention of the full sequence (the pages' dense
+ *   branch for layers outside the sparse set): Qh = Q [B,L,H,d], Kh = K and
+ *   Vh = V [B,L,Hkv,d], Oh = O [B,L,H,d]; Lkeep is ignored and may be NULL.
+ * scale > 0 (normally 1/sqrt(d)).  ws supplies the error word. */
+TSA_API tsa_status tsa_attn(const tsa_dims *dims, const void *Qh, const void *Kh, const void *Vh,
+                    const int32_t *Lkeep, int32_t dense, float scale, void *Oh,
+                    void *ws, size_t ws_bytes, void *stream);
+
+/* Decompress and residual ([notes] 关键设计 1: X_{l+1} = X_l + Decompress(Ô), unselected
+ * rows of the decompressed tensor are zero; [blog] §1.1 解压缩阶段; [gist] §2
+ * Decompression).
+ *   idx != NULL: Y[b, idx[b,h,i], h*d:(h+1)*d] = X[...] + Oh[b,h,i] for i < Lkeep[b].
+ *     If Y != X, every other segment gets Y = X; this reads the complement that
+ *     tsa_select stores in idx[b,h,Lkeep[b]:L].  If Y == X the update is in place
+ *     and only the kept segments are touched.
+ *   idx == NULL: dense layer, Oh is O [B,L,H,d] and Y = X + O (Lkeep ignored).
+ * The sum is formed in fp32 and rounded once to the output type.  Y may equal X;
+ * no other aliasing is allowed. */
+TSA_API tsa_status tsa_scatter_residual(const tsa_dims *dims, const void *Oh, const int32_t *idx,
+                                const int32_t *Lkeep, const void *X, void *Y, void *stream);
+
+/* The whole layer ([notes] 整体框架): is_sparse != 0 runs tsa_score, tsa_budget,
+ * tsa_select, tsa_gather_qkv, tsa_attn and tsa_scatter_residual in order with no host
+ * synchronisation; is_sparse == 0 runs dense causal attention and the residual (the
+ * dense branch for layers outside the sparse set; which layers are sparse is the
+ * caller's input).  s_h_out, s_l_out, Lkeep_out, idx_out are optional (NULL: kept in
+ * ws); when given they receive those intermediates.  stage_events, if not NULL,
+ * points to 7 cudaEvent_t (as void*) recorded before scoring and after each of the
+ * six stages (for a dense layer the first five are recorded at the start).
+ * Y may equal X. */
+TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const void *V,
+                     const void *X, void *Y, int32_t is_sparse, int32_t q, double tau,
+                     float scale, float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
+                     int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
+                     void *const *stage_events);
+
+/* Synchronises `stream`, returns the device error word recorded in `ws` (TSA_OK if
+ * none) and clears it. */
+TSA_API tsa_status tsa_get_device_status(void *ws, void *stream);
+
+/* Upper bound, in spin iterations, of every device-side wait in later launches
+ * (default 2^26).  Tests lower it to check that a wait that runs out is reported
+ * as TSA_ERR_DEVICE_TIMEOUT instead of hanging. */
+TSA_API void tsa_set_wait_limit(uint32_t iterations);
+
+TSA_API const char *tsa_status_string(tsa_status s);
+TSA_API const char *tsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TSA_H_ */

@@ -1,0 +1,347 @@
+// C ABI of libtsa: argument checks, workspace layout, stage dispatch and the fused layer.
+// Every entry point only enqueues kernels on the caller's stream.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "common.cuh"
+
+namespace tsa {
+
+cudaError_t launch_score_simt(const tsa_dims &, const void *, const void *, int, float, float *,
+                              const WsLayout &, char *, cudaStream_t);
+cudaError_t launch_score_tc(const tsa_dims &, const void *, const void *, int, float, float *,
+                            const WsLayout &, char *, cudaStream_t, uint32_t);
+cudaError_t launch_norm(const tsa_dims &, const float *, float *, const WsLayout &, char *,
+                        cudaStream_t);
+cudaError_t launch_budget(const tsa_dims &, const float *, double, int32_t *, Control *,
+                          cudaStream_t);
+cudaError_t launch_select(const tsa_dims &, const float *, const int32_t *, int32_t *,
+                          Control *, cudaStream_t);
+cudaError_t launch_gather(const tsa_dims &, const void *, const void *, const void *,
+                          const int32_t *, const int32_t *, void *, void *, void *, cudaStream_t);
+cudaError_t launch_attn_simt(const tsa_dims &, const void *, const void *, const void *,
+                             const int32_t *, int, float, void *, cudaStream_t);
+cudaError_t launch_attn_tc(const tsa_dims &, const void *, const void *, const void *,
+                           const int32_t *, int, float, void *, Control *, cudaStream_t,
+                           uint32_t);
+cudaError_t launch_scatter(const tsa_dims &, const void *, const int32_t *, const int32_t *,
+                           const void *, void *, cudaStream_t);
+
+static thread_local std::string g_last_error;
+static uint32_t g_wait_limit = 1u << 26;
+
+static tsa_status fail(tsa_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+static tsa_status cuda_status(cudaError_t e, const char *where) {
+    if (e == cudaSuccess) return TSA_OK;
+    return fail(TSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define TSA_TRY(expr)                        \
+    do {                                     \
+        const tsa_status s_ = (expr);        \
+        if (s_ != TSA_OK) return s_;         \
+    } while (0)
+
+static size_t esize(const tsa_dims &dm) { return dm.dtype == TSA_F32 ? 4 : 2; }
+
+static tsa_status check_dims(const tsa_dims *dm) {
+    if (!dm) return fail(TSA_ERR_INVALID_ARG, "dims is NULL");
+    if (dm->B < 1 || dm->L < 1 || dm->H < 1 || dm->Hkv < 1)
+        return fail(TSA_ERR_INVALID_ARG, "B, L, H, Hkv must be >= 1 (got %d, %d, %d, %d)",
+                    dm->B, dm->L, dm->H, dm->Hkv);
+    if (dm->L > (1 << 21)) return fail(TSA_ERR_UNSUPPORTED, "L = %d exceeds 2^21", dm->L);
+    if (dm->H % dm->Hkv) return fail(TSA_ERR_INVALID_ARG, "H %% Hkv != 0 (%d, %d)", dm->H, dm->Hkv);
+    if (dm->d != 64 && dm->d != 128) return fail(TSA_ERR_UNSUPPORTED, "d = %d (64 or 128)", dm->d);
+    if (dm->dtype != TSA_F32 && dm->dtype != TSA_BF16)
+        return fail(TSA_ERR_UNSUPPORTED, "dtype %d", dm->dtype);
+    if ((long long)dm->B * dm->H * dm->L > (1ll << 31))
+        return fail(TSA_ERR_UNSUPPORTED, "B*H*L exceeds 2^31");
+    return TSA_OK;
+}
+
+static tsa_status check_q(const tsa_dims *dm, int q) {
+    if (q < 1) return fail(TSA_ERR_INVALID_ARG, "q = %d must be >= 1", q);
+    const int qe = q < dm->L ? q : dm->L;
+    if ((dm->H / dm->Hkv) * qe > 256)
+        return fail(TSA_ERR_UNSUPPORTED, "G * min(q, L) = %d exceeds 256", (dm->H / dm->Hkv) * qe);
+    return TSA_OK;
+}
+
+static tsa_status check_ptr(const void *p, const char *name) {
+    if (!p) return fail(TSA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) & 15)
+        return fail(TSA_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
+    return TSA_OK;
+}
+
+static tsa_status check_scale(float scale) {
+    if (!(scale > 0.0f) || !isfinite(scale))
+        return fail(TSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+    return TSA_OK;
+}
+
+WsLayout ws_layout(const tsa_dims &dm, int q) {
+    WsLayout w;
+    w.qe = q < dm.L ? q : dm.L;
+    w.N = (dm.H / dm.Hkv) * w.qe;
+    w.nsplit = ceil_div(dm.L, kScoreSplitTokens);
+    w.nblk_norm = ceil_div(dm.L, 256);
+    size_t off = align256(sizeof(Control));
+    w.score_part = off;
+    off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.nsplit * w.N);
+    w.score_stat = off;
+    off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.N);
+    w.norm_part = off;
+    off = align256(off + sizeof(float) * (size_t)dm.B * w.nblk_norm);
+    w.total = off;
+    return w;
+}
+
+struct LayerLayout {
+    size_t s_h, s_l, lkeep, idx, qh, kh, vh, oh, total;
+};
+
+static LayerLayout layer_layout(const tsa_dims &dm, int q) {
+    LayerLayout y;
+    size_t off = ws_layout(dm, q).total;
+    const size_t BHL = (size_t)dm.B * dm.H * dm.L;
+    y.s_h = off; off = align256(off + 4 * BHL);
+    y.s_l = off; off = align256(off + 4 * (size_t)dm.B * dm.L);
+    y.lkeep = off; off = align256(off + 4 * (size_t)dm.B);
+    y.idx = off; off = align256(off + 4 * BHL);
+    const size_t t = align256(BHL * dm.d * esize(dm));
+    y.qh = off; off += t;
+    y.kh = off; off += t;
+    y.vh = off; off += t;
+    y.oh = off; off += t;
+    y.total = off;
+    return y;
+}
+
+static tsa_status check_ws(const void *ws, size_t have, size_t need) {
+    if (!ws) return fail(TSA_ERR_WORKSPACE, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255)
+        return fail(TSA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+    if (have < need)
+        return fail(TSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", have, need);
+    return TSA_OK;
+}
+
+// ---------------------------------------------------------------- stages ---
+
+static tsa_status do_score(const tsa_dims &dm, const void *Q, const void *K, int q, float scale,
+                           float *s_h, float *s_l, char *ws, cudaStream_t st) {
+    const WsLayout w = ws_layout(dm, q);
+    cudaError_t e;
+    e = launch_score_simt(dm, Q, K, w.qe, scale, s_h, w, ws, st);
+    TSA_TRY(cuda_status(e, "tsa_score"));
+    return cuda_status(launch_norm(dm, s_h, s_l, w, ws, st), "tsa_score (normalise)");
+}
+
+static tsa_status do_attn(const tsa_dims &dm, const void *Q, const void *K, const void *V,
+                          const int32_t *Lkeep, int dense, float scale, void *O, char *ws,
+                          cudaStream_t st) {
+    cudaError_t e;
+    e = launch_attn_simt(dm, Q, K, V, Lkeep, dense, scale, O, st);
+    (void)ws;
+    return cuda_status(e, "tsa_attn");
+}
+
+}  // namespace tsa
+
+using namespace tsa;
+
+extern "C" {
+
+size_t tsa_workspace_size(const tsa_dims *dims, int32_t q) {
+    if (check_dims(dims) != TSA_OK || check_q(dims, q) != TSA_OK) return 0;
+    return ws_layout(*dims, q).total;
+}
+
+size_t tsa_layer_workspace_size(const tsa_dims *dims, int32_t q) {
+    if (check_dims(dims) != TSA_OK || check_q(dims, q) != TSA_OK) return 0;
+    return layer_layout(*dims, q).total;
+}
+
+tsa_status tsa_score(const tsa_dims *dims, const void *Q, const void *K, int32_t q, float scale,
+                     float *s_h, float *s_l, void *ws, size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_q(dims, q));
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_ptr(Q, "Q"));
+    TSA_TRY(check_ptr(K, "K"));
+    TSA_TRY(check_ptr(s_h, "s_h"));
+    TSA_TRY(check_ptr(s_l, "s_l"));
+    TSA_TRY(check_ws(ws, ws_bytes, ws_layout(*dims, q).total));
+    return do_score(*dims, Q, K, q, scale, s_h, s_l, (char *)ws, (cudaStream_t)stream);
+}
+
+tsa_status tsa_budget(const tsa_dims *dims, const float *s_l, double tau, int32_t *Lkeep,
+                      void *ws, size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    if (!(tau >= 0.0 && tau < 1.0)) return fail(TSA_ERR_INVALID_ARG, "tau must be in [0, 1)");
+    TSA_TRY(check_ptr(s_l, "s_l"));
+    TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
+    return cuda_status(launch_budget(*dims, s_l, tau, Lkeep, (Control *)ws, (cudaStream_t)stream),
+                       "tsa_budget");
+}
+
+tsa_status tsa_select(const tsa_dims *dims, const float *s_h, const int32_t *Lkeep, int32_t *idx,
+                      void *ws, size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_ptr(s_h, "s_h"));
+    TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    TSA_TRY(check_ptr(idx, "idx"));
+    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
+    return cuda_status(
+        launch_select(*dims, s_h, Lkeep, idx, (Control *)ws, (cudaStream_t)stream), "tsa_select");
+}
+
+tsa_status tsa_gather_qkv(const tsa_dims *dims, const void *Q, const void *K, const void *V,
+                          const int32_t *idx, const int32_t *Lkeep, void *Qh, void *Kh, void *Vh,
+                          void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_ptr(Q, "Q"));
+    TSA_TRY(check_ptr(K, "K"));
+    TSA_TRY(check_ptr(V, "V"));
+    TSA_TRY(check_ptr(idx, "idx"));
+    TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    TSA_TRY(check_ptr(Qh, "Qh"));
+    TSA_TRY(check_ptr(Kh, "Kh"));
+    TSA_TRY(check_ptr(Vh, "Vh"));
+    return cuda_status(
+        launch_gather(*dims, Q, K, V, idx, Lkeep, Qh, Kh, Vh, (cudaStream_t)stream),
+        "tsa_gather_qkv");
+}
+
+tsa_status tsa_attn(const tsa_dims *dims, const void *Qh, const void *Kh, const void *Vh,
+                    const int32_t *Lkeep, int32_t dense, float scale, void *Oh, void *ws,
+                    size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_ptr(Qh, "Qh"));
+    TSA_TRY(check_ptr(Kh, "Kh"));
+    TSA_TRY(check_ptr(Vh, "Vh"));
+    TSA_TRY(check_ptr(Oh, "Oh"));
+    if (!dense) TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
+    return do_attn(*dims, Qh, Kh, Vh, Lkeep, dense ? 1 : 0, scale, Oh, (char *)ws,
+                   (cudaStream_t)stream);
+}
+
+tsa_status tsa_scatter_residual(const tsa_dims *dims, const void *Oh, const int32_t *idx,
+                                const int32_t *Lkeep, const void *X, void *Y, void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_ptr(Oh, "Oh"));
+    TSA_TRY(check_ptr(X, "X"));
+    TSA_TRY(check_ptr(Y, "Y"));
+    if (idx) {
+        TSA_TRY(check_ptr(idx, "idx"));
+        TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    }
+    return cuda_status(launch_scatter(*dims, Oh, idx, Lkeep, X, Y, (cudaStream_t)stream),
+                       "tsa_scatter_residual");
+}
+
+tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const void *V,
+                     const void *X, void *Y, int32_t is_sparse, int32_t q, double tau,
+                     float scale, float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
+                     int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
+                     void *const *stage_events) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_q(dims, q));
+    TSA_TRY(check_scale(scale));
+    if (!(tau >= 0.0 && tau < 1.0)) return fail(TSA_ERR_INVALID_ARG, "tau must be in [0, 1)");
+    TSA_TRY(check_ptr(Q, "Q"));
+    TSA_TRY(check_ptr(K, "K"));
+    TSA_TRY(check_ptr(V, "V"));
+    TSA_TRY(check_ptr(X, "X"));
+    TSA_TRY(check_ptr(Y, "Y"));
+    for (const void *p : {(const void *)s_h_out, (const void *)s_l_out, (const void *)Lkeep_out,
+                          (const void *)idx_out})
+        if (p) TSA_TRY(check_ptr(p, "optional output"));
+    const tsa_dims &dm = *dims;
+    const LayerLayout y = layer_layout(dm, q);
+    TSA_TRY(check_ws(ws, ws_bytes, y.total));
+    char *w = (char *)ws;
+    cudaStream_t st = (cudaStream_t)stream;
+    auto rec = [&](int i) -> tsa_status {
+        if (!stage_events) return TSA_OK;
+        return cuda_status(cudaEventRecord((cudaEvent_t)stage_events[i], st), "event record");
+    };
+    float *s_h = s_h_out ? s_h_out : (float *)(w + y.s_h);
+    float *s_l = s_l_out ? s_l_out : (float *)(w + y.s_l);
+    int32_t *Lk = Lkeep_out ? Lkeep_out : (int32_t *)(w + y.lkeep);
+    int32_t *idx = idx_out ? idx_out : (int32_t *)(w + y.idx);
+    void *Qh = w + y.qh, *Kh = w + y.kh, *Vh = w + y.vh, *Oh = w + y.oh;
+    if (!is_sparse) {
+        for (int i = 0; i < 5; ++i) TSA_TRY(rec(i));
+        TSA_TRY(do_attn(dm, Q, K, V, nullptr, 1, scale, Oh, w, st));
+        TSA_TRY(rec(5));
+        TSA_TRY(cuda_status(launch_scatter(dm, Oh, nullptr, nullptr, X, Y, st), "tsa_layer"));
+        return rec(6);
+    }
+    TSA_TRY(rec(0));
+    TSA_TRY(do_score(dm, Q, K, q, scale, s_h, s_l, w, st));
+    TSA_TRY(rec(1));
+    TSA_TRY(cuda_status(launch_budget(dm, s_l, tau, Lk, (Control *)w, st), "tsa_layer budget"));
+    TSA_TRY(rec(2));
+    TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, (Control *)w, st), "tsa_layer select"));
+    TSA_TRY(rec(3));
+    TSA_TRY(cuda_status(launch_gather(dm, Q, K, V, idx, Lk, Qh, Kh, Vh, st), "tsa_layer gather"));
+    TSA_TRY(rec(4));
+    TSA_TRY(do_attn(dm, Qh, Kh, Vh, Lk, 0, scale, Oh, w, st));
+    TSA_TRY(rec(5));
+    TSA_TRY(cuda_status(launch_scatter(dm, Oh, idx, Lk, X, Y, st), "tsa_layer scatter"));
+    return rec(6);
+}
+
+tsa_status tsa_get_device_status(void *ws, void *stream) {
+    if (!ws) return fail(TSA_ERR_WORKSPACE, "workspace is NULL");
+    cudaStream_t st = (cudaStream_t)stream;
+    TSA_TRY(cuda_status(cudaStreamSynchronize(st), "tsa_get_device_status"));
+    Control c;
+    TSA_TRY(cuda_status(cudaMemcpy(&c, ws, sizeof c, cudaMemcpyDeviceToHost),
+                        "tsa_get_device_status read"));
+    if (c.err != 0) {
+        const int32_t zero[2] = {0, 0};
+        TSA_TRY(cuda_status(cudaMemcpy(ws, zero, sizeof zero, cudaMemcpyHostToDevice),
+                            "tsa_get_device_status clear"));
+        return fail((tsa_status)c.err, "device error %d (detail %d)", c.err, c.err_where);
+    }
+    return TSA_OK;
+}
+
+void tsa_set_wait_limit(uint32_t iterations) { g_wait_limit = iterations; }
+
+const char *tsa_status_string(tsa_status s) {
+    switch (s) {
+        case TSA_OK: return "TSA_OK";
+        case TSA_ERR_INVALID_ARG: return "TSA_ERR_INVALID_ARG";
+        case TSA_ERR_ALIGNMENT: return "TSA_ERR_ALIGNMENT";
+        case TSA_ERR_UNSUPPORTED: return "TSA_ERR_UNSUPPORTED";
+        case TSA_ERR_WORKSPACE: return "TSA_ERR_WORKSPACE";
+        case TSA_ERR_CUDA: return "TSA_ERR_CUDA";
+        case TSA_ERR_DEVICE_TIMEOUT: return "TSA_ERR_DEVICE_TIMEOUT";
+        case TSA_ERR_NONFINITE: return "TSA_ERR_NONFINITE";
+    }
+    return "TSA_ERR_UNKNOWN";
+}
+
+const char *tsa_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

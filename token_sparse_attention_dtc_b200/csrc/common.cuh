@@ -1,0 +1,65 @@
+// Shared device/host helpers of the CUDA library (not used by the CPU oracle).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tsa.h"
+
+namespace tsa {
+
+// Workspace control block: the first 256 bytes of every workspace.
+struct Control {
+    int32_t err;        // first device error (tsa_status), 0 when none
+    int32_t err_where;  // kernel-specific detail of that error
+    int32_t pad[62];
+};
+static_assert(sizeof(Control) == 256, "control block is 256 bytes");
+
+constexpr int kScoreSplitTokens = 4096;  // tokens per scoring split (SIMT path)
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Device error reporting: the first error wins.
+__device__ inline void report_error(Control *c, int code, int where) {
+    if (atomicCAS(&c->err, 0, code) == 0) c->err_where = where;
+}
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ inline float load(const float *p, size_t i) { return p[i]; }
+    static __device__ inline float to_f(float x) { return x; }
+    static __device__ inline float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ inline float load(const __nv_bfloat16 *p, size_t i) {
+        return __bfloat162float(p[i]);
+    }
+    static __device__ inline float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ inline __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// Scores are non-negative floats: their IEEE bits order like the values.  -0.0 maps
+// to +0.0; anything negative, above 1, infinite or NaN is flagged.
+__device__ inline uint32_t score_key(float v, bool &bad) {
+    uint32_t k = __float_as_uint(v);
+    if (k == 0x80000000u) k = 0;
+    if (k > 0x3f800000u) { bad = true; k = 0; }
+    return k;
+}
+
+// Layout of the workspace regions used by the stage kernels.
+struct WsLayout {
+    size_t control = 0;     // Control
+    size_t score_part = 0;  // float2 [B*Hkv][nsplit][N]  per-split (max, sum) in log2 units
+    size_t score_stat = 0;  // float2 [B*Hkv][N]          combined (max, 1/sum)
+    size_t norm_part = 0;   // float  [B][nblk]            partial sums of u
+    size_t total = 0;
+    int nsplit = 0, N = 0, qe = 0, nblk_norm = 0;
+};
+
+WsLayout ws_layout(const tsa_dims &dm, int q);
+
+}  // namespace tsa

@@ -1,0 +1,220 @@
+"""Python binding of libtsa: the same entry points as include/tsa.h.
+
+Argument marshalling only: tensors become device pointers, torch's current
+stream becomes the stream argument, and a non-OK status becomes a TSAError.
+Every step of the layer runs in the CUDA library; if libtsa.so is missing the
+first call raises instead of doing anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtsa.so")
+_lib = None
+
+TSA_F32, TSA_BF16 = 0, 1
+STATUS = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_ALIGNMENT",
+          3: "TSA_ERR_UNSUPPORTED", 4: "TSA_ERR_WORKSPACE", 5: "TSA_ERR_CUDA",
+          6: "TSA_ERR_DEVICE_TIMEOUT", 7: "TSA_ERR_NONFINITE"}
+EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_budget",
+           "tsa_select", "tsa_gather_qkv", "tsa_attn", "tsa_scatter_residual", "tsa_layer",
+           "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
+           "tsa_last_error")
+
+
+class TSAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__("%s: %s" % (STATUS.get(status, status), msg))
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+def lib():
+    """Load libtsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError("libtsa.so is not built (python -m token_sparse_attention_dtc_b200.build)")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I32, SZ, D, F = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_double,
+                            ctypes.c_float)
+        DP = ctypes.POINTER(Dims)
+        sig = {
+            "tsa_workspace_size": (SZ, [DP, I32]),
+            "tsa_layer_workspace_size": (SZ, [DP, I32]),
+            "tsa_score": (I32, [DP, P, P, I32, F, P, P, P, SZ, P]),
+            "tsa_budget": (I32, [DP, P, D, P, P, SZ, P]),
+            "tsa_select": (I32, [DP, P, P, P, P, SZ, P]),
+            "tsa_gather_qkv": (I32, [DP, P, P, P, P, P, P, P, P, P]),
+            "tsa_attn": (I32, [DP, P, P, P, P, I32, F, P, P, SZ, P]),
+            "tsa_scatter_residual": (I32, [DP, P, P, P, P, P, P]),
+            "tsa_layer": (I32, [DP, P, P, P, P, P, I32, I32, D, F, P, P, P, P, P, SZ, P, P]),
+            "tsa_get_device_status": (I32, [P, P]),
+            "tsa_set_wait_limit": (None, [ctypes.c_uint32]),
+            "tsa_status_string": (ctypes.c_char_p, [I32]),
+            "tsa_last_error": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise TSAError(status, lib().tsa_last_error().decode())
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def dims(Q: torch.Tensor, K: torch.Tensor) -> Dims:
+    """Dims of Q [B, L, H, d] and K [B, L, Hkv, d]."""
+    B, L, H, d = Q.shape
+    if Q.dtype == torch.bfloat16:
+        dt = TSA_BF16
+    elif Q.dtype == torch.float32:
+        dt = TSA_F32
+    else:
+        raise ValueError("Q must be bf16 or fp32")
+    return Dims(B, L, H, K.shape[2], d, dt)
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)
+
+
+def workspace_size(dm: Dims, q: int, layer: bool = False) -> int:
+    f = lib().tsa_layer_workspace_size if layer else lib().tsa_workspace_size
+    n = f(ctypes.byref(dm), q)
+    if n == 0:
+        raise TSAError(1, lib().tsa_last_error().decode())
+    return n
+
+
+def workspace(dm: Dims, q: int, layer: bool = False, device=None) -> torch.Tensor:
+    """A zero-filled workspace (torch allocations are 256-byte aligned)."""
+    return torch.zeros(workspace_size(dm, q, layer), dtype=torch.uint8, device=device or "cuda")
+
+
+def tsa_score(Q, K, q: int, scale: float | None = None, s_h=None, s_l=None, ws=None,
+              stream=None):
+    dm = dims(Q, K)
+    _need_cuda(Q, K)
+    if s_h is None:
+        s_h = torch.empty(dm.B, dm.H, dm.L, dtype=torch.float32, device=Q.device)
+    if s_l is None:
+        s_l = torch.empty(dm.B, dm.L, dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = workspace(dm, q, device=Q.device)
+    _check(lib().tsa_score(ctypes.byref(dm), _p(Q), _p(K), q,
+                           default_scale(dm.d) if scale is None else scale, _p(s_h), _p(s_l),
+                           _p(ws), ws.numel(), _stream(stream)))
+    return s_h, s_l
+
+
+def tsa_budget(dm: Dims, s_l, tau: float, Lkeep=None, ws=None, stream=None):
+    _need_cuda(s_l)
+    if Lkeep is None:
+        Lkeep = torch.empty(dm.B, dtype=torch.int32, device=s_l.device)
+    if ws is None:
+        ws = workspace(dm, 1, device=s_l.device)
+    _check(lib().tsa_budget(ctypes.byref(dm), _p(s_l), float(tau), _p(Lkeep), _p(ws),
+                            ws.numel(), _stream(stream)))
+    return Lkeep
+
+
+def tsa_select(dm: Dims, s_h, Lkeep, idx=None, ws=None, stream=None):
+    _need_cuda(s_h, Lkeep)
+    if idx is None:
+        idx = torch.empty(dm.B, dm.H, dm.L, dtype=torch.int32, device=s_h.device)
+    if ws is None:
+        ws = workspace(dm, 1, device=s_h.device)
+    _check(lib().tsa_select(ctypes.byref(dm), _p(s_h), _p(Lkeep), _p(idx), _p(ws), ws.numel(),
+                            _stream(stream)))
+    return idx
+
+
+def tsa_gather_qkv(Q, K, V, idx, Lkeep, Qh=None, Kh=None, Vh=None, stream=None):
+    dm = dims(Q, K)
+    _need_cuda(Q, K, V, idx, Lkeep)
+    shape = (dm.B, dm.H, dm.L, dm.d)
+    Qh = torch.empty(shape, dtype=Q.dtype, device=Q.device) if Qh is None else Qh
+    Kh = torch.empty(shape, dtype=Q.dtype, device=Q.device) if Kh is None else Kh
+    Vh = torch.empty(shape, dtype=Q.dtype, device=Q.device) if Vh is None else Vh
+    _check(lib().tsa_gather_qkv(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(idx), _p(Lkeep),
+                                _p(Qh), _p(Kh), _p(Vh), _stream(stream)))
+    return Qh, Kh, Vh
+
+
+def tsa_attn(dm: Dims, Qh, Kh, Vh, Lkeep=None, dense: bool = False, scale: float | None = None,
+             Oh=None, ws=None, stream=None):
+    _need_cuda(Qh, Kh, Vh, Lkeep)
+    if Oh is None:
+        Oh = torch.empty_like(Qh)
+    if ws is None:
+        ws = workspace(dm, 1, device=Qh.device)
+    _check(lib().tsa_attn(ctypes.byref(dm), _p(Qh), _p(Kh), _p(Vh), _p(Lkeep), int(dense),
+                          default_scale(dm.d) if scale is None else scale, _p(Oh), _p(ws),
+                          ws.numel(), _stream(stream)))
+    return Oh
+
+
+def tsa_scatter_residual(dm: Dims, Oh, idx, Lkeep, X, Y=None, stream=None):
+    _need_cuda(Oh, idx, Lkeep, X)
+    if Y is None:
+        Y = torch.empty_like(X)
+    _check(lib().tsa_scatter_residual(ctypes.byref(dm), _p(Oh), _p(idx), _p(Lkeep), _p(X),
+                                      _p(Y), _stream(stream)))
+    return Y
+
+
+def tsa_layer(Q, K, V, X, Y=None, is_sparse: bool = True, q: int = 16, tau: float = 0.005,
+              scale: float | None = None, s_h=None, s_l=None, Lkeep=None, idx=None, ws=None,
+              stream=None, stage_events=None):
+    """One Token Sparse Attention layer: returns Y = X + Decompress(Ô) (or the dense layer)."""
+    dm = dims(Q, K)
+    _need_cuda(Q, K, V, X, Y, s_h, s_l, Lkeep, idx)
+    if Y is None:
+        Y = torch.empty_like(X)
+    if ws is None:
+        ws = workspace(dm, q, layer=True, device=Q.device)
+    ev = None
+    if stage_events is not None:
+        ev = (ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
+    _check(lib().tsa_layer(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y), int(is_sparse),
+                           q, float(tau), default_scale(dm.d) if scale is None else scale,
+                           _p(s_h), _p(s_l), _p(Lkeep), _p(idx), _p(ws), ws.numel(),
+                           _stream(stream), ev))
+    return Y
+
+
+def tsa_get_device_status(ws, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    st = lib().tsa_get_device_status(_p(ws), _stream(stream))
+    return int(st)
+
+
+def tsa_set_wait_limit(iterations: int):
+    lib().tsa_set_wait_limit(int(iterations))
