@@ -1,0 +1,402 @@
+"""Benchmark of the Token Sparse Attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama8b_128k] [--no-dense] [--no-e2e] [--no-cpu-baseline]
+
+A step is one sparse layer (score, budget, select, gather, attention, scatter +
+residual) on one sequence of the workload, inputs resident in HBM.  Prints one JSON
+line on rank 0.  With N > 1 (torchrun) every rank runs its own sequence (batch
+sharded, no collective on the data path): weak scaling, time = max over ranks.
+
+--impl reference times the CPU oracle (the fp64 restatement of the pages' method) on
+the host cores, each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "token-sparse attn layer ms @128K Llama-8B shape; TFLOP/s & % roofline"
+STAGES = ("score", "budget", "select", "gather", "attn", "scatter")
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sus=d.get("bf16_tflops_sustained", d["bf16_tflops"]), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def _traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e:
+        return None
+    import hashlib
+
+    src = os.path.join(ROOT, "token_sparse_attention_dtc_b200", "csrc", e["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return e["bytes_per_launch"] if h == e["source_sha"] else None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                rows.append((float(f[0]), float(f[1]), f[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i] == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "samples": len(rows), "reasons": reasons}
+
+
+def _workload_desc(w, L):
+    return ("%s: B=1 per GPU, L=%d, H=%d, Hkv=%d, d=%d, bf16, q=%d, tau=%g, 4 sinks + "
+            "%.1f%% heavy hitters shifted %.1f along per-group query directions"
+            % (w.name, L, w.H, w.Hkv, w.d, w.q, w.tau, 100 * w.heavy_frac, w.shift))
+
+
+# --------------------------------------------------------------------------- oracle ---
+
+def oracle_sample(x, w, L, rows_per_sample=64, slice_div=64):
+    """Time the oracle on a bounded sample of one layer; return (ms per full layer, info)."""
+    import numpy as np
+
+    import oracle
+
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    s_h, s_l = oracle.score(x["Q"], x["K"], w.q, nthreads=threads)
+    t1 = time.perf_counter()
+    lk, _ = oracle.budget(s_l.astype(np.float32), w.tau)
+    t2 = time.perf_counter()
+    idx = oracle.select(s_h.astype(np.float32), lk)
+    t3 = time.perf_counter()
+    Lk = int(lk[0])
+    # attention: rows of head 0 spread over [0, L'), extrapolated by exact causal pair count
+    rows_i = sorted(set(np.linspace(0, max(Lk - 1, 0), rows_per_sample).astype(int).tolist()))
+    rows = [(0, 0, i) for i in rows_i] if Lk else []
+    ta = time.perf_counter()
+    if rows:
+        oracle.attend_rows(x["Q"], x["K"], x["V"], idx, lk, rows, nthreads=threads)
+    tb = time.perf_counter()
+    pairs_sample = sum(i + 1 for i in rows_i) if rows else 1
+    pairs_full = w.H * Lk * (Lk + 1) / 2
+    t_attn = (tb - ta) * pairs_full / pairs_sample if rows else 0.0
+    # decompress + residual on 1/slice_div of the tokens, scaled by token count
+    n = max(1, L // slice_div)
+    Oh = np.zeros((1, w.H, n, w.d))
+    idx_s = np.tile(np.arange(n, dtype=np.int32), (1, w.H, 1))
+    tc = time.perf_counter()
+    oracle.decompress_residual(Oh, idx_s, np.array([min(Lk, n)], np.int32), x["X"][:, :n])
+    td = time.perf_counter()
+    t_dec = (td - tc) * L / n
+    total = (t1 - t0) + (t2 - t1) + (t3 - t2) + t_attn + t_dec
+    info = dict(score_s=t1 - t0, budget_s=t2 - t1, select_s=t3 - t2,
+                attn_s_extrapolated=t_attn, attn_rows_sampled=len(rows),
+                decompress_s_extrapolated=t_dec, Lkeep=Lk, threads=threads)
+    sample = ("full scoring, budget and selection on the %d-token sequence; attention on %d "
+              "query rows of head 0 extrapolated to all %d heads by causal pair count; "
+              "decompress+residual on %d tokens scaled by token count"
+              % (L, len(rows), w.H, n))
+    return total * 1e3, sample, info, (tb - ta) + (t1 - t0) + (t2 - t1) + (t3 - t2) + (td - tc)
+
+
+def run_reference(args, w, L, rank, world):
+    if rank != 0:
+        return
+    from token_sparse_attention_dtc_b200.inputs import make_workload
+
+    x = make_workload(w.name, seed=args.seed, L=L, B=1)
+    times = []
+    sample = info = None
+    for s in range(args.warmup + args.steps):
+        ms, sample, info, _ = oracle_sample(x, w, L)
+        if s >= args.warmup:
+            times.append(ms)
+    v = statistics.mean(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "ms", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": v,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": _workload_desc(w, L), "oracle": "fp64 C, pthreads"},
+        "cpu_baseline": {"value": v, "unit": "ms", "cores": info["threads"], "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "oracle_breakdown_s": info,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- ours ---
+
+def run_ours(args, w, L, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from token_sparse_attention_dtc_b200 import tsa
+    from token_sparse_attention_dtc_b200.inputs import make_workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    tsa.lib()  # fail loudly if the CUDA library is missing
+    x = make_workload(w.name, seed=args.seed * 1000 + rank, L=L, B=1)
+    d = {k: v.to(dev) for k, v in x.items()}
+    dm = tsa.dims(d["Q"], d["K"])
+    ws = tsa.workspace(dm, w.q, layer=True, device=dev)
+    Y = torch.empty_like(d["X"])
+    Lk = torch.empty(1, dtype=torch.int32, device=dev)
+    st = torch.cuda.current_stream(dev)
+
+    def sync_all():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    n_ev = 7
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+           for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(st)  # materialise the event handles
+    for _ in range(args.warmup):
+        tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk, ws=ws)
+    sync_all()
+    if tsa.tsa_get_device_status(ws) != 0:
+        raise RuntimeError("device error during warm-up")
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        time.sleep(0.3)
+        sync_all()
+        t_start.record(st)
+        for s in range(args.steps):
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk, ws=ws,
+                          stage_events=evs[s])
+        t_stop.record(st)
+        sync_all()
+    total_ms = t_start.elapsed_time(t_stop)
+    ms_step = total_ms / args.steps
+    stage_ms = {name: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1])
+                                      for s in range(args.steps))
+                for i, name in enumerate(STAGES)}
+    lk = int(Lk.item())
+    if tsa.tsa_get_device_status(ws) != 0:
+        raise RuntimeError("device error during the timed region")
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    peaks = _peaks()
+    flops = 2.0 * w.H * w.d * lk * (lk + 1)
+    attn_ms = stage_ms["attn"]
+    attn_tf = flops / (attn_ms * 1e-3) / 1e12
+    roof = {"kernel": "k_attn_tc", "bound": "tensor", "achieved": attn_tf,
+            "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_sus"],
+            "peak_kind": "bf16 sustained (%s)" % peaks["src"],
+            "frac_of_burst": attn_tf / peaks["bf16"],
+            "traffic": _traffic("k_attn_tc", w.name)}
+    # HBM kernels: algorithmic bytes per launch
+    H, dd = w.H, w.d
+    hbm = {
+        "score": (L * w.Hkv * dd * 2 + w.q * H * dd * 2 + 4 * H * L + 4 * L),
+        "gather": 6 * H * lk * dd * 2,
+        "scatter": 2 * L * H * dd * 2 + H * lk * dd * 2 + 4 * H * L,
+    }
+    hbm_roof = {k: {"ms": stage_ms[k], "achieved_gbs": v / (stage_ms[k] * 1e-3) / 1e9,
+                    "frac": v / (stage_ms[k] * 1e-3) / 1e9 / peaks["hbm"],
+                    "algorithmic_bytes": v}
+                for k, v in hbm.items()}
+
+    # dense causal attention through the same kernel, same shape
+    dense = None
+    if not args.no_dense:
+        for _ in range(2):
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, is_sparse=False, ws=ws)
+        dev_ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+        for e in dev_ev:
+            e.record(st)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        sync_all()
+        a.record(st)
+        nd = 2
+        for _ in range(nd):
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, is_sparse=False, ws=ws,
+                          stage_events=dev_ev)
+        b.record(st)
+        sync_all()
+        dms = a.elapsed_time(b) / nd
+        dflops = 2.0 * w.H * w.d * L * (L + 1)
+        dattn = dev_ev[4].elapsed_time(dev_ev[5])
+        dense = {"layer_ms": dms, "attn_ms": dattn,
+                 "attn_tflops": dflops / (dattn * 1e-3) / 1e12,
+                 "attn_frac_of_sustained": dflops / (dattn * 1e-3) / 1e12 / peaks["bf16_sus"],
+                 "speedup_sparse_vs_dense_layer": dms / ms_step}
+
+    # end to end through the public API with host buffers (copies inside the timed region)
+    e2e = None
+    if not args.no_e2e:
+        hx = {k: v.pin_memory() for k, v in x.items()}
+        hY = torch.empty(x["X"].shape, dtype=x["X"].dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hx.values())
+        d2h = hY.numel() * hY.element_size()
+
+        def e2e_step():
+            for k in d:
+                d[k].copy_(hx[k], non_blocking=True)
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, ws=ws)
+            hY.copy_(Y, non_blocking=True)
+
+        e2e_step()
+        sync_all()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        ne = max(1, min(args.steps, 3))
+        sync_all()
+        a.record(st)
+        for _ in range(ne):
+            e2e_step()
+        b.record(st)
+        sync_all()
+        ems = a.elapsed_time(b) / ne
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": ems / world, "unit": "ms", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": ne}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms, sample, info, _ = oracle_sample(x, w, L)
+        cpu = {"value": ms, "unit": "ms", "cores": info["threads"], "kind": "oracle",
+               "sample": sample}
+
+    launches_per_step = 10  # score: 3 + 2 (normalise), budget, select, gather, attn, scatter
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": ms_step / world, "unit": "ms", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": _workload_desc(w, L), "global_batch": world, "seq_len": L,
+                       "parallelism": "replicas (dp%d, no data-path collective)" % world,
+                       "l2": "inputs larger than L2 (Q 1.07 GB, K/V 268 MB each); no flush",
+                       "Lkeep": lk, "kept_fraction": lk / L},
+            "roofline": roof,
+            "stages_ms": stage_ms,
+            "hbm_kernels": hbm_roof,
+            "attn_tflops": attn_tf,
+            "layer_tflops": flops / (ms_step * 1e-3) / 1e12,
+            "overhead_fraction": 1.0 - attn_ms / sum(stage_ms.values()),
+            "dense": dense,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": clk.summary(),
+            "gpu_launches": launches_per_step * args.steps,
+            "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--workload", default="llama8b_128k")
+    ap.add_argument("--L", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+
+    from token_sparse_attention_dtc_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    L = args.L or w.L
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":  # rank 0 alone times the oracle; other ranks exit
+        run_reference(args, w, L, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, w, L, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -59,7 +59,7 @@ typedef enum {
     TSA_ERR_WORKSPACE = 4,      /* workspace too small or misaligned              */
     TSA_ERR_CUDA = 5,           /* a CUDA runtime or launch error                 */
     TSA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait ran out             */
-    TSA_ERR_NONFINITE = 7       /* a score outside [0, 1] or not finite           */
+    TSA_ERR_NONFINITE = 7       /* s_l outside [0, 1], s_h < 0, or a NaN / inf score */
 } tsa_status;
 
 typedef enum { TSA_F32 = 0, TSA_BF16 = 1 } tsa_dtype;
@@ -166,10 +166,11 @@ TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K,
  * none) and clears it. */
 TSA_API tsa_status tsa_get_device_status(void *ws, void *stream);
 
-/* Upper bound, in spin iterations, of every device-side wait in later launches
- * (default 2^26).  Tests lower it to check that a wait that runs out is reported
- * as TSA_ERR_DEVICE_TIMEOUT instead of hanging. */
-TSA_API void tsa_set_wait_limit(uint32_t iterations);
+/* Upper bound, in microseconds, of every device-side wait (on an mbarrier) in later
+ * launches from any thread; default 2 000 000 (2 s).  A wait that runs out makes its
+ * kernel record TSA_ERR_DEVICE_TIMEOUT, finish the copies and MMAs it started, free its
+ * tensor memory and exit; tests lower the limit to check that path. */
+TSA_API void tsa_set_wait_limit(uint32_t microseconds);
 
 TSA_API const char *tsa_status_string(tsa_status s);
 TSA_API const char *tsa_last_error(void);

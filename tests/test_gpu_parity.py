@@ -305,3 +305,21 @@ def test_headline_128k_sampled():
     for (t, seg), o in zip(where, vals):
         ref = Xd[0, t, seg] + o
         assert np.all(np.abs(Yd[0, t, seg] - ref) <= 2e-2 + 2.0 ** -8 * np.abs(ref))
+
+
+def test_attention_is_deterministic():
+    """Repeated launches on the same inputs give bit-identical outputs (no races)."""
+    x = _dev(make_workload("llama8b_4k", seed=2))
+    dm = tsa.dims(x["Q"], x["K"])
+    ws = tsa.workspace(dm, 16)
+    s_h, s_l = tsa.tsa_score(x["Q"], x["K"], 16, ws=ws)
+    Lk = tsa.tsa_budget(dm, s_l, 0.005, ws=ws)
+    idx = tsa.tsa_select(dm, s_h, Lk, ws=ws)
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(x["Q"], x["K"], x["V"], idx, Lk)
+    lk = int(Lk.item())
+    ref = tsa.tsa_attn(dm, Qh, Kh, Vh, Lk, ws=ws)[:, :, :lk].clone()
+    refd = tsa.tsa_attn(dm, x["Q"], x["K"], x["V"], None, dense=True, ws=ws).clone()
+    for _ in range(8):
+        assert torch.equal(tsa.tsa_attn(dm, Qh, Kh, Vh, Lk, ws=ws)[:, :, :lk], ref)
+        assert torch.equal(tsa.tsa_attn(dm, x["Q"], x["K"], x["V"], None, dense=True, ws=ws), refd)
+    assert tsa.tsa_get_device_status(ws) == 0

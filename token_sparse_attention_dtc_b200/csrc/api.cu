@@ -32,7 +32,7 @@ cudaError_t launch_scatter(const tsa_dims &, const void *, const int32_t *, cons
                            const void *, void *, cudaStream_t);
 
 static thread_local std::string g_last_error;
-static uint32_t g_wait_limit = 1u << 26;
+static uint32_t g_wait_limit_us = 2000000;  // 2 s
 
 static tsa_status fail(tsa_status s, const char *fmt, ...) {
     char buf[512];
@@ -155,8 +155,11 @@ static tsa_status do_attn(const tsa_dims &dm, const void *Q, const void *K, cons
                           const int32_t *Lkeep, int dense, float scale, void *O, char *ws,
                           cudaStream_t st) {
     cudaError_t e;
-    e = launch_attn_simt(dm, Q, K, V, Lkeep, dense, scale, O, st);
-    (void)ws;
+    if (dm.dtype == TSA_BF16)
+        e = launch_attn_tc(dm, Q, K, V, Lkeep, dense, scale, O, reinterpret_cast<Control *>(ws),
+                           st, g_wait_limit_us);
+    else
+        e = launch_attn_simt(dm, Q, K, V, Lkeep, dense, scale, O, st);
     return cuda_status(e, "tsa_attn");
 }
 
@@ -326,7 +329,7 @@ tsa_status tsa_get_device_status(void *ws, void *stream) {
     return TSA_OK;
 }
 
-void tsa_set_wait_limit(uint32_t iterations) { g_wait_limit = iterations; }
+void tsa_set_wait_limit(uint32_t microseconds) { g_wait_limit_us = microseconds; }
 
 const char *tsa_status_string(tsa_status s) {
     switch (s) {

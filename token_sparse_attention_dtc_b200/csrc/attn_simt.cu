@@ -1,5 +1,6 @@
 // Causal attention on CUDA cores for fp32 inputs (the fp32 path keeps full fp32
-// products; tensor-core tf32 would not meet a 1e-4 output tolerance).  Flash-style
+// products; tensor-core tf32 would not meet a 1e-4 output tolerance).  bf16 inputs run on
+// the tensor cores (attn_tc.cu).  Flash-style
 // online softmax over 64-key tiles, one block per (64-row query tile, batch, head).
 //
 // Method: "Token Sparse Attention" papernotes.org notes, 整体框架 (dense attention on
@@ -134,12 +135,9 @@ static cudaError_t attn_simt_impl(const tsa_dims &dm, const void *Q, const void 
 cudaError_t launch_attn_simt(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                              const int32_t *Lkeep, int dense, float scale, void *O,
                              cudaStream_t st) {
-    if (dm.dtype == TSA_F32)
-        return dm.d == 64 ? attn_simt_impl<float, 64>(dm, Q, K, V, Lkeep, dense, scale, O, st)
-                          : attn_simt_impl<float, 128>(dm, Q, K, V, Lkeep, dense, scale, O, st);
-    return dm.d == 64
-               ? attn_simt_impl<__nv_bfloat16, 64>(dm, Q, K, V, Lkeep, dense, scale, O, st)
-               : attn_simt_impl<__nv_bfloat16, 128>(dm, Q, K, V, Lkeep, dense, scale, O, st);
+    if (dm.dtype != TSA_F32) return cudaErrorInvalidValue;  // bf16 runs on the tensor cores
+    return dm.d == 64 ? attn_simt_impl<float, 64>(dm, Q, K, V, Lkeep, dense, scale, O, st)
+                      : attn_simt_impl<float, 128>(dm, Q, K, V, Lkeep, dense, scale, O, st);
 }
 
 }  // namespace tsa

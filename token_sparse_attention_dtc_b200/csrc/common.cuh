@@ -42,13 +42,17 @@ template <> struct Elem<__nv_bfloat16> {
 };
 
 // Scores are non-negative floats: their IEEE bits order like the values.  -0.0 maps
-// to +0.0; anything negative, above 1, infinite or NaN is flagged.
+// to +0.0; a value above `max_bits` (the bits of the largest legal score), a negative
+// value, an infinity or a NaN is flagged and treated as 0.
+template <uint32_t max_bits>
 __device__ inline uint32_t score_key(float v, bool &bad) {
     uint32_t k = __float_as_uint(v);
     if (k == 0x80000000u) k = 0;
-    if (k > 0x3f800000u) { bad = true; k = 0; }
+    if (k > max_bits) { bad = true; k = 0; }
     return k;
 }
+constexpr uint32_t kLayerScoreMax = 0x3f800000u;  // s_l <= 1
+constexpr uint32_t kHeadScoreMax = 0x7f7fffffu;   // s_h <= q: any finite non-negative
 
 // Layout of the workspace regions used by the stage kernels.
 struct WsLayout {

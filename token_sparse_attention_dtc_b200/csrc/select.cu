@@ -11,7 +11,6 @@
 namespace tsa {
 
 constexpr int kSelThreads = 1024;
-constexpr int kSelWarps = kSelThreads / 32;
 
 // Fixed-point mass of one score: floor(v * 2^62), exact for v in [0, 1].
 __device__ inline unsigned long long mass62(uint32_t key) {
@@ -41,7 +40,7 @@ k_budget(const float *__restrict__ s_l, int L, unsigned long long T, int32_t *__
         __syncthreads();
         const uint32_t prefix = s_prefix, mask = s_mask;
         for (int t = threadIdx.x; t < L; t += blockDim.x) {
-            const uint32_t key = score_key(s[t], bad);
+            const uint32_t key = score_key<kLayerScoreMax>(s[t], bad);
             if ((key & mask) == prefix) {
                 const int dg = (key >> shift) & 255;
                 atomicAdd(&cnt[dg], 1u);
@@ -134,7 +133,7 @@ k_select(const float *__restrict__ s_h, int L, int H, const int32_t *__restrict_
         __syncthreads();
         const uint32_t prefix = s_prefix, mask = s_mask;
         for (int t = threadIdx.x; t < L; t += blockDim.x) {
-            const uint32_t key = score_key(s[t], bad);
+            const uint32_t key = score_key<kHeadScoreMax>(s[t], bad);
             if ((key & mask) == prefix) atomicAdd(&cnt[(key >> shift) & 255], 1u);
         }
         __syncthreads();
@@ -156,7 +155,7 @@ k_select(const float *__restrict__ s_h, int L, int H, const int32_t *__restrict_
     for (int t0 = 0; t0 < L; t0 += blockDim.x) {
         const int t = t0 + threadIdx.x;
         bool dummy = false;
-        const uint32_t key = t < L ? score_key(s[t], dummy) : 0u;
+        const uint32_t key = t < L ? score_key<kHeadScoreMax>(s[t], dummy) : 0u;
         const bool eq = t < L && key == thr;
         int n_eq;
         const int eq_rank = base_eq + block_scan_flag(eq, warp_tot, n_eq);
