@@ -162,6 +162,29 @@ TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K,
                      int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
                      void *const *stage_events);
 
+/* Scoring for callers that cannot allocate device memory when they call in, such as an
+ * engine whose device memory is fully planned up front by its own allocator, or a host
+ * thread that must not enter the CUDA allocator.  Those callers cannot create the `ws`
+ * tsa_score needs.  The pages have no counterpart: this is tsa_score (same arguments
+ * minus the workspace, same kernels, same results) with its scratch taken from a fixed
+ * 2 MiB array in the library's device image, held on every GPU that loads the library
+ * until the process exits.  The caller still passes Q, K, s_h and s_l.
+ *   Limit   dims and q whose scoring workspace (tsa_workspace_size) exceeds 2 MiB are
+ *           rejected with TSA_ERR_WORKSPACE before any device work; for example
+ *           B = 1, L = 131072, 32/8 heads, q = 16 needs about 140 KB.
+ *   Set-up  the first call on each device looks up the array's device address (with
+ *           that device current) and caches it; make that first call before any stream
+ *           capture.
+ *   Sharing every call on a device uses the same array, which keeps the last call's
+ *           contents (the call clears the part that must start at zero).  Calls whose
+ *           work overlaps on the GPU (other streams, or other host threads) race on it
+ *           and must be serialised by the caller.  Device-side errors of this call are
+ *           not readable through tsa_get_device_status.
+ * It allocates and frees nothing. */
+TSA_API tsa_status tsa_score_fixed_scratch(const tsa_dims *dims, const void *Q, const void *K,
+                                           int32_t q, float scale, float *s_h, float *s_l,
+                                           void *stream);
+
 /* Synchronises `stream`, returns the device error word recorded in `ws` (TSA_OK if
  * none) and clears it. */
 TSA_API tsa_status tsa_get_device_status(void *ws, void *stream);

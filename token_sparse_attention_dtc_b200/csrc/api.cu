@@ -44,6 +44,11 @@ static tsa_status fail(tsa_status s, const char *fmt, ...) {
     return s;
 }
 
+tsa_status set_error(tsa_status s, const char *msg) {
+    g_last_error = msg;
+    return s;
+}
+
 static tsa_status cuda_status(cudaError_t e, const char *where) {
     if (e == cudaSuccess) return TSA_OK;
     return fail(TSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));

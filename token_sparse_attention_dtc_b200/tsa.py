@@ -23,7 +23,7 @@ STATUS = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_ALIGNMENT",
 EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_budget",
            "tsa_select", "tsa_gather_qkv", "tsa_attn", "tsa_scatter_residual", "tsa_layer",
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
-           "tsa_last_error")
+           "tsa_last_error", "tsa_score_fixed_scratch")
 
 
 class TSAError(RuntimeError):
@@ -61,6 +61,7 @@ def lib():
             "tsa_set_wait_limit": (None, [ctypes.c_uint32]),
             "tsa_status_string": (ctypes.c_char_p, [I32]),
             "tsa_last_error": (ctypes.c_char_p, []),
+            "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -131,6 +132,22 @@ def tsa_score(Q, K, q: int, scale: float | None = None, s_h=None, s_l=None, ws=N
     _check(lib().tsa_score(ctypes.byref(dm), _p(Q), _p(K), q,
                            default_scale(dm.d) if scale is None else scale, _p(s_h), _p(s_l),
                            _p(ws), ws.numel(), _stream(stream)))
+    return s_h, s_l
+
+
+def tsa_score_fixed_scratch(Q, K, q: int, scale: float | None = None, s_h=None, s_l=None,
+                            stream=None):
+    """tsa_score without a workspace argument: the library's fixed device scratch is used
+    (for callers that cannot allocate device memory at call time)."""
+    dm = dims(Q, K)
+    _need_cuda(Q, K)
+    if s_h is None:
+        s_h = torch.empty(dm.B, dm.H, dm.L, dtype=torch.float32, device=Q.device)
+    if s_l is None:
+        s_l = torch.empty(dm.B, dm.L, dtype=torch.float32, device=Q.device)
+    _check(lib().tsa_score_fixed_scratch(ctypes.byref(dm), _p(Q), _p(K), q,
+                                         default_scale(dm.d) if scale is None else scale,
+                                         _p(s_h), _p(s_l), _stream(stream)))
     return s_h, s_l
 
 
