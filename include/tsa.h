@@ -171,7 +171,7 @@ TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K,
  * until the process exits.  The caller still passes Q, K, s_h and s_l.
  *   Limit   dims and q whose scoring workspace (tsa_workspace_size) exceeds 2 MiB are
  *           rejected with TSA_ERR_WORKSPACE before any device work; for example
- *           B = 1, L = 131072, 32/8 heads, q = 16 needs about 140 KB.
+ *           B = 1, L = 131072, 32/8 heads, q = 16 needs about 240 KB.
  *   Set-up  the first call on each device looks up the array's device address (with
  *           that device current) and caches it; make that first call before any stream
  *           capture.

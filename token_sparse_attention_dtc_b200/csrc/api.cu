@@ -5,6 +5,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <string>
 
 #include "common.cuh"
@@ -17,7 +18,7 @@ cudaError_t launch_score_tc(const tsa_dims &, const void *, const void *, int, f
                             const WsLayout &, char *, cudaStream_t, uint32_t);
 cudaError_t launch_norm(const tsa_dims &, const float *, float *, const WsLayout &, char *,
                         cudaStream_t);
-cudaError_t launch_budget(const tsa_dims &, const float *, double, int32_t *, Control *,
+cudaError_t launch_budget(const tsa_dims &, const float *, double, int32_t *, char *,
                           cudaStream_t);
 cudaError_t launch_select(const tsa_dims &, const float *, const int32_t *, int32_t *,
                           Control *, cudaStream_t);
@@ -102,9 +103,11 @@ WsLayout ws_layout(const tsa_dims &dm, int q) {
     WsLayout w;
     w.qe = q < dm.L ? q : dm.L;
     w.N = (dm.H / dm.Hkv) * w.qe;
-    w.nsplit = ceil_div(dm.L, kScoreSplitTokens);
+    // splits per KV group: the CUDA-core path uses ceil(L / 4096), the tensor-core path
+    // at most min(#128-token tiles, 256)
+    w.nsplit = std::max(ceil_div(dm.L, kScoreSplitTokens), std::min(ceil_div(dm.L, 128), 256));
     w.nblk_norm = ceil_div(dm.L, 256);
-    size_t off = align256(sizeof(Control));
+    size_t off = budget_end(dm.B);  // control block, budget state and histograms first
     w.score_part = off;
     off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.nsplit * w.N);
     w.score_stat = off;
@@ -151,7 +154,10 @@ static tsa_status do_score(const tsa_dims &dm, const void *Q, const void *K, int
                            float *s_h, float *s_l, char *ws, cudaStream_t st) {
     const WsLayout w = ws_layout(dm, q);
     cudaError_t e;
-    e = launch_score_simt(dm, Q, K, w.qe, scale, s_h, w, ws, st);
+    if (dm.dtype == TSA_BF16)
+        e = launch_score_tc(dm, Q, K, w.qe, scale, s_h, w, ws, st, g_wait_limit_us);
+    else
+        e = launch_score_simt(dm, Q, K, w.qe, scale, s_h, w, ws, st);
     TSA_TRY(cuda_status(e, "tsa_score"));
     return cuda_status(launch_norm(dm, s_h, s_l, w, ws, st), "tsa_score (normalise)");
 }
@@ -203,8 +209,8 @@ tsa_status tsa_budget(const tsa_dims *dims, const float *s_l, double tau, int32_
     if (!(tau >= 0.0 && tau < 1.0)) return fail(TSA_ERR_INVALID_ARG, "tau must be in [0, 1)");
     TSA_TRY(check_ptr(s_l, "s_l"));
     TSA_TRY(check_ptr(Lkeep, "Lkeep"));
-    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
-    return cuda_status(launch_budget(*dims, s_l, tau, Lkeep, (Control *)ws, (cudaStream_t)stream),
+    TSA_TRY(check_ws(ws, ws_bytes, budget_end(dims->B)));
+    return cuda_status(launch_budget(*dims, s_l, tau, Lkeep, (char *)ws, (cudaStream_t)stream),
                        "tsa_budget");
 }
 
@@ -306,7 +312,7 @@ tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const v
     TSA_TRY(rec(0));
     TSA_TRY(do_score(dm, Q, K, q, scale, s_h, s_l, w, st));
     TSA_TRY(rec(1));
-    TSA_TRY(cuda_status(launch_budget(dm, s_l, tau, Lk, (Control *)w, st), "tsa_layer budget"));
+    TSA_TRY(cuda_status(launch_budget(dm, s_l, tau, Lk, w, st), "tsa_layer budget"));
     TSA_TRY(rec(2));
     TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, (Control *)w, st), "tsa_layer select"));
     TSA_TRY(rec(3));

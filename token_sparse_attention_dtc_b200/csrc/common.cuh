@@ -54,6 +54,27 @@ __device__ inline uint32_t score_key(float v, bool &bad) {
 constexpr uint32_t kLayerScoreMax = 0x3f800000u;  // s_l <= 1
 constexpr uint32_t kHeadScoreMax = 0x7f7fffffu;   // s_h <= q: any finite non-negative
 
+// Coverage-budget search state of one batch element (workspace, after the control block).
+struct BudgetState {
+    uint32_t prefix;            // key digits chosen so far
+    int32_t done;               // 1 once k is known
+    int32_t k;                  // tokens pruned (valid when done)
+    int32_t cbefore;            // count of scores below the current digit range
+    unsigned long long before;  // their fixed-point mass
+    unsigned long long pad;
+};
+static_assert(sizeof(BudgetState) == 32, "budget state is 32 bytes");
+constexpr size_t kBudgetStateOffset = 256;
+// Per batch element: two 4096-digit levels and one 256-digit level of (uint32 count,
+// uint64 mass).
+constexpr size_t kBudgetHistBytes = 4096 * 12 * 2 + 256 * 12;
+__host__ __device__ inline size_t budget_hist_offset(int B) {
+    return align256(kBudgetStateOffset + sizeof(BudgetState) * (size_t)B);
+}
+__host__ __device__ inline size_t budget_end(int B) {
+    return align256(budget_hist_offset(B) + kBudgetHistBytes * (size_t)B);
+}
+
 // Layout of the workspace regions used by the stage kernels.
 struct WsLayout {
     size_t control = 0;     // Control

@@ -1,5 +1,7 @@
-// Dynamic Token Coverage scoring on CUDA cores (fp32 inputs), plus the layer-score
-// normalisation shared by every dtype.
+// Dynamic Token Coverage scoring on CUDA cores for fp32 inputs (tf32 tensor cores would
+// not meet the 1e-5 score tolerance; bf16 inputs score on the tensor cores in
+// score_tc.cu), the split combine, and the layer-score normalisation shared by every
+// dtype.
 //
 // Method: "Token Sparse Attention" papernotes.org notes, 关键设计 2 (recent queries
 // score all keys; column sums give s_h; their normalised sum gives s_l); bxzpzcl.cn
@@ -235,12 +237,15 @@ static cudaError_t score_simt_impl(const tsa_dims &dm, const void *Q, const void
 cudaError_t launch_score_simt(const tsa_dims &dm, const void *Q, const void *K, int qe,
                               float scale, float *s_h, const WsLayout &w, char *ws,
                               cudaStream_t st) {
-    if (dm.dtype == TSA_F32)
-        return dm.d == 64 ? score_simt_impl<float, 64>(dm, Q, K, qe, scale, s_h, w, ws, st)
-                          : score_simt_impl<float, 128>(dm, Q, K, qe, scale, s_h, w, ws, st);
-    return dm.d == 64
-               ? score_simt_impl<__nv_bfloat16, 64>(dm, Q, K, qe, scale, s_h, w, ws, st)
-               : score_simt_impl<__nv_bfloat16, 128>(dm, Q, K, qe, scale, s_h, w, ws, st);
+    if (dm.dtype != TSA_F32) return cudaErrorInvalidValue;  // bf16 scores on the tensor cores
+    return dm.d == 64 ? score_simt_impl<float, 64>(dm, Q, K, qe, scale, s_h, w, ws, st)
+                      : score_simt_impl<float, 128>(dm, Q, K, qe, scale, s_h, w, ws, st);
+}
+
+cudaError_t launch_combine(const float2 *part, int nsplit, int N, float2 *stat, int groups,
+                           cudaStream_t st) {
+    k_score_combine<<<groups, 256, 0, st>>>(part, nsplit, N, stat);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_norm(const tsa_dims &dm, const float *s_h, float *s_l, const WsLayout &w,

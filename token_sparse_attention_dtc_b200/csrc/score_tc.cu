@@ -1,0 +1,352 @@
+// Dynamic Token Coverage scoring on the tensor cores (bf16 inputs), exact two-pass softmax.
+//
+// Method: "Token Sparse Attention" papernotes.org notes, 关键设计 2 (the last q queries
+// score all keys with a per-head softmax; column sums give s_h); bxzpzcl.cn post §2.1;
+// gist.science §2 "Scoring".  For KV group kv the N = G*qe recent-query rows of its G
+// heads (row n = g*qe + i -> head kv*G+g, position L-qe+i) are scored against 128-token
+// K tiles.  All logits are z2 = scale*log2(e)*<q, k> in fp32 (bf16 products, fp32
+// accumulation in TMEM).
+//
+// Pass 1 (k_score_stats_tc): S = Qblk · Ktile^T with the query rows on the TMEM lanes
+//   (M = 128 query rows, zero-padded; two row blocks when N > 128), 128 tokens per MMA.
+//   Each epilogue thread owns one query row and keeps its running (max, sum of 2^(z2-max))
+//   over the CTA's contiguous token range, so no cross-thread reduction is needed; the
+//   CTA writes one (max, sum) per row.  k_score_combine (score_simt.cu) merges the splits.
+// Pass 2 (k_score_colsum_tc): S^T = Ktile · Qblk^T with the tokens on the TMEM lanes
+//   (M = 128 tokens, N = query rows padded to 16).  Each thread owns one token and adds
+//   2^(z2 - max_n) / sum_n over the rows n of each head in row order, then stores
+//   s_h[b, h, t].  The CTA walks its token range backwards, so its first tiles are the
+//   ones pass 1 read last (likely still in L2).
+// Both passes: warp 0 streams K tiles by TMA through a 4-stage ring, warp 1 issues the
+// MMAs into two TMEM accumulators, warps 4-7 run the epilogue.  All waits are bounded.
+#include <math.h>
+
+#include <algorithm>
+
+#include "sm100.cuh"
+
+namespace tsa {
+using namespace sm100;
+
+namespace {
+
+constexpr int kThreads = 256, kStages = 4, kTile = 128;
+constexpr uint64_t kDrainNs = 1000000000ull;
+
+template <int D> struct ScoreSmem {
+    static constexpr int KT = kTile * D * 2;  // bytes of one K tile
+    alignas(1024) uint8_t q[2 * 128 * D * 2];  // up to 256 query rows, swizzled, K-major
+    alignas(1024) uint8_t k[kStages][KT];
+    uint64_t k_full[kStages], k_empty[kStages], acc_full[2], acc_empty[2], drain;
+    float2 stat[256];  // pass 2: (max, 1/sum) per query row
+    uint32_t tmem_base;
+    int abort, never;
+};
+
+// Copy the N recent-query rows of group (b, kv) into shared memory in the 128-byte swizzled
+// K-major layout the MMA descriptors expect; rows N..nrows-1 are zero.
+template <int D>
+__device__ inline void load_q_block(uint8_t *qs, const __nv_bfloat16 *__restrict__ Q, int b,
+                                    int kv, int L, int H, int G, int qe, int N, int nrows) {
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    const int block_bytes = nrows * 128;
+    for (int e = threadIdx.x; e < nrows * CPR; e += kThreads) {
+        const int n = e / CPR, ch = e % CPR;
+        const int db = ch / 8, c8 = ch % 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < N) {
+            const int g = n / qe, i = n % qe;
+            const size_t off = (((size_t)b * L + (L - qe + i)) * H + kv * G + g) * D + ch * 8;
+            v = *reinterpret_cast<const uint4 *>(Q + off);
+        }
+        *reinterpret_cast<uint4 *>(qs + db * block_bytes + n * 128 + ((c8 ^ (n & 7)) * 16)) = v;
+    }
+}
+
+// Tile range [first, first + count) of this CTA among the group's ntiles tiles.
+__device__ inline void tile_range(int ntiles, int nsplit, int split, int &first, int &count) {
+    const int per = ntiles / nsplit, rem = ntiles % nsplit;
+    first = split * per + min(split, rem);
+    count = per + (split < rem ? 1 : 0);
+}
+
+template <int D, bool kPass2>
+__global__ void __launch_bounds__(kThreads, 1)
+k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restrict__ Q, int L,
+           int H, int Hkv, int qe, float sl2, int nsplit, float2 *__restrict__ part,
+           const float2 *__restrict__ stat, float *__restrict__ s_h, Control *ctl,
+           uint64_t limit_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    ScoreSmem<D> &sm = *reinterpret_cast<ScoreSmem<D> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int KT = ScoreSmem<D>::KT, NDB = D / 64;
+    const int split = blockIdx.x, bg = blockIdx.y;
+    const int b = bg / Hkv, kv = bg % Hkv, G = H / Hkv, N = G * qe;
+    const int RB = (N + 127) / 128;              // pass 1 row blocks
+    const int Npad = (N + 15) & ~15;             // pass 2 MMA N
+    const int nrows = kPass2 ? Npad : RB * 128;  // query rows held in shared memory
+    const int ntiles = (L + kTile - 1) / kTile;
+    int first, count;
+    tile_range(ntiles, nsplit, split, first, count);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&sm.acc_full[a], 1);
+            mbar_init(&sm.acc_empty[a], 128);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        sm.never = 0;
+        fence_mbar_init();
+    }
+    load_q_block<D>(sm.q, Q, b, kv, L, H, G, qe, N, nrows);
+    if (kPass2)
+        for (int n = threadIdx.x; n < N; n += kThreads) sm.stat[n] = stat[(size_t)bg * N + n];
+    fence_proxy_async_smem();  // make the generic-proxy Q writes visible to the MMA
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t acc_cols = kPass2 ? 256u : (uint32_t)RB * 128u;  // per accumulator
+    volatile int *abort = &sm.abort;
+    bool ok = true;
+    // Order of tiles: pass 1 ascending, pass 2 descending within the CTA's range.
+    auto tile_at = [&](int it) { return kPass2 ? first + count - 1 - it : first + it; };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int it = 0; it < count; ++it) {
+                const int s = it % kStages;
+                if (!(ok = mbar_wait(&sm.k_empty[s], ((it / kStages) & 1) ^ 1, limit_ns, abort)))
+                    break;
+                mbar_expect_tx(&sm.k_full[s], KT);
+#pragma unroll
+                for (int db = 0; db < NDB; ++db)
+                    tma_load_4d(sm.k[s] + db * kTile * 128, &tmK, &sm.k_full[s], db * 64,
+                                tile_at(it) * kTile, kv, b);
+                issued = it + 1;
+            }
+            for (int it = (issued > kStages ? issued - kStages : 0); it < issued; ++it)
+                mbar_wait(&sm.k_full[it % kStages], (it / kStages) & 1, kDrainNs, &sm.never);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t qa = smem_u32(sm.q);
+            const uint32_t id1 = idesc_bf16(128, kTile, false);
+            const uint32_t id2 = idesc_bf16(128, Npad, false);
+            bool any = false;
+            for (int it = 0; it < count; ++it) {
+                const int s = it % kStages, a = it & 1;
+                if (!(ok = mbar_wait(&sm.k_full[s], (it / kStages) & 1, limit_ns, abort))) break;
+                if (!(ok = mbar_wait(&sm.acc_empty[a], ((it >> 1) & 1) ^ 1, limit_ns, abort)))
+                    break;
+                tc_fence_after();
+                const uint32_t ka = smem_u32(sm.k[s]);
+                const uint32_t dacc = tmem + a * acc_cols;
+                if (!kPass2) {
+                    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t kof = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
+                            const uint32_t qof = (kk / 4) * (nrows * 128) + rb * 128 * 128 + (kk % 4) * 32;
+                            mma_ss(dacc + rb * 128, sdesc_sw128(qa + qof, 16, 1024),
+                                   sdesc_sw128(ka + kof, 16, 1024), id1, kk > 0 ? 1u : 0u);
+                        }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t kof = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
+                        const uint32_t qof = (kk / 4) * (nrows * 128) + (kk % 4) * 32;
+                        mma_ss(dacc, sdesc_sw128(ka + kof, 16, 1024),
+                               sdesc_sw128(qa + qof, 16, 1024), id2, kk > 0 ? 1u : 0u);
+                    }
+                }
+                any = true;
+                mma_commit(&sm.k_empty[s]);
+                mma_commit(&sm.acc_full[a]);
+            }
+            if (any) {
+                mma_commit(&sm.drain);
+                mbar_wait(&sm.drain, 0, kDrainNs, &sm.never);
+            }
+        }
+    } else if (warp >= 4) {
+        const int wq = warp & 3, r = wq * 32 + lane;
+        const uint32_t lo = (uint32_t)(wq * 32) << 16;
+        const int pmin = L - qe;  // first recent-query position
+        if (!kPass2) {
+            // thread r owns query rows r (+128 for a second row block)
+            float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
+            int pr[2];
+            for (int rb = 0; rb < 2; ++rb) {
+                const int n = rb * 128 + r;
+                pr[rb] = n < N ? L - qe + (n % qe) : -1;  // -1: padding row, never valid
+            }
+            for (int it = 0; it < count; ++it) {
+                const int a = it & 1;
+                ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                const int t0 = tile_at(it) * kTile;
+                const bool tail = t0 + kTile - 1 > pmin;  // some token may follow a query
+                for (int rb = 0; rb < RB; ++rb) {
+                    if (rb * 128 + wq * 32 >= N) continue;  // whole warp on padding rows
+#pragma unroll
+                    for (int c = 0; c < kTile / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + a * acc_cols + rb * 128 + c * 32 + lo, v);
+                        tmem_ld_wait();
+                        if (pr[rb] < 0) continue;
+                        float cm = -INFINITY;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            float z = __uint_as_float(v[e]);
+                            if (tail && t0 + c * 32 + e > pr[rb]) z = -INFINITY;
+                            v[e] = __float_as_uint(z);
+                            cm = fmaxf(cm, z);
+                        }
+                        if (cm == -INFINITY) continue;
+                        cm *= sl2;
+                        if (cm > m[rb]) {
+                            l[rb] = (m[rb] == -INFINITY) ? 0.0f : l[rb] * ex2(m[rb] - cm);
+                            m[rb] = cm;
+                        }
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            acc += ex2(fmaf(__uint_as_float(v[e]), sl2, -m[rb]));
+                        l[rb] += acc;
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.acc_empty[a]);
+            }
+            if (ok)
+                for (int rb = 0; rb < RB; ++rb) {
+                    const int n = rb * 128 + r;
+                    if (n < N) part[((size_t)bg * nsplit + split) * N + n] = make_float2(m[rb], l[rb]);
+                }
+        } else {
+            const int nchunks = Npad / 32 + ((Npad % 32) ? 1 : 0);
+            for (int it = 0; it < count; ++it) {
+                const int a = it & 1;
+                ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                const int t = tile_at(it) * kTile + r;
+                int g = 0, i = 0;
+                float acc = 0.0f;
+                for (int c = 0; c < nchunks; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + a * acc_cols + c * 32 + lo, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int n = c * 32 + e;
+                        if (n >= N) break;
+                        const float2 st = sm.stat[n];
+                        if (t <= pmin + i)
+                            acc = fmaf(ex2(fmaf(__uint_as_float(v[e]), sl2, -st.x)), st.y, acc);
+                        if (++i == qe) {
+                            if (t < L) s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
+                            acc = 0.0f;
+                            i = 0;
+                            ++g;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.acc_empty[a]);
+            }
+        }
+    }
+    if (!ok) {
+        *abort = 1;
+        report_error(ctl, TSA_ERR_DEVICE_TIMEOUT, (kPass2 ? 300 : 200) + warp);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+    }
+    return n;
+}
+
+}  // namespace
+
+// Splits per KV group of the tensor-core scoring: about one CTA per SM in total.
+int score_tc_splits(const tsa_dims &dm) {
+    const int ntiles = ceil_div(dm.L, kTile);
+    return std::max(1, std::min(ntiles, std::min(256, sm_count() / std::max(1, dm.B * dm.Hkv))));
+}
+
+cudaError_t launch_combine(const float2 *part, int nsplit, int N, float2 *stat, int groups,
+                           cudaStream_t st);
+
+template <int D>
+static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *K, int qe,
+                                 float scale, float *s_h, const WsLayout &w, char *ws,
+                                 cudaStream_t st, uint32_t limit_us) {
+    CUtensorMap tk;
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)dm.L, (uint64_t)dm.Hkv, (uint64_t)dm.B};
+    const uint64_t strides[3] = {(uint64_t)dm.Hkv * D * 2, (uint64_t)D * 2,
+                                 (uint64_t)dm.L * dm.Hkv * D * 2};
+    const uint32_t box[4] = {64, (uint32_t)kTile, 1, 1};
+    if (!make_tmap_bf16_4d(&tk, K, dims, strides, box)) return cudaErrorInvalidValue;
+    // At least 116 KB so that one CTA holds an SM (and all 512 TMEM columns) at a time.
+    const size_t smem = std::max<size_t>(sizeof(ScoreSmem<D>) + 1024, 116 * 1024);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k_score_tc<D, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+        return e;
+    if ((e = cudaFuncSetAttribute(k_score_tc<D, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+        return e;
+    const int nsplit = score_tc_splits(dm);
+    const float sl2 = scale * 1.4426950408889634f;
+    float2 *part = reinterpret_cast<float2 *>(ws + w.score_part);
+    float2 *stat = reinterpret_cast<float2 *>(ws + w.score_stat);
+    Control *ctl = reinterpret_cast<Control *>(ws);
+    const uint64_t lim = (uint64_t)limit_us * 1000ull;
+    dim3 grid(nsplit, dm.B * dm.Hkv);
+    k_score_tc<D, false><<<grid, kThreads, smem, st>>>(tk, (const __nv_bfloat16 *)Q, dm.L, dm.H,
+                                                       dm.Hkv, qe, sl2, nsplit, part, stat,
+                                                       s_h, ctl, lim);
+    if ((e = cudaGetLastError())) return e;
+    const int N = (dm.H / dm.Hkv) * qe;
+    if ((e = launch_combine(part, nsplit, N, stat, dm.B * dm.Hkv, st))) return e;
+    k_score_tc<D, true><<<grid, kThreads, smem, st>>>(tk, (const __nv_bfloat16 *)Q, dm.L, dm.H,
+                                                      dm.Hkv, qe, sl2, nsplit, part, stat,
+                                                      s_h, ctl, lim);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_score_tc(const tsa_dims &dm, const void *Q, const void *K, int qe,
+                            float scale, float *s_h, const WsLayout &w, char *ws,
+                            cudaStream_t st, uint32_t limit_us) {
+    return dm.d == 64 ? score_tc_impl<64>(dm, Q, K, qe, scale, s_h, w, ws, st, limit_us)
+                      : score_tc_impl<128>(dm, Q, K, qe, scale, s_h, w, ws, st, limit_us);
+}
+
+}  // namespace tsa

@@ -1,86 +1,14 @@
-// Coverage budget and per-head top-L' selection: block-wide radix selection over the
-// IEEE bits of the (non-negative) fp32 scores, with integer histograms only, so the
-// results do not depend on thread scheduling.
+// Per-head top-L' selection: block-wide radix selection over the IEEE bits of the
+// (non-negative) fp32 head scores, with integer histograms only, so the results do not
+// depend on thread scheduling; then an ordered compaction.
 //
-// Method: "Token Sparse Attention" papernotes.org notes, 关键设计 2 (sort s_l
-// ascending, smallest k whose cumulative mass reaches tau, keep L - k; each head
-// keeps its own top-k_keep); bxzpzcl.cn post §2.1 层级预算分配; gist.science §2
-// "Budget Allocation" and "Head-Wise Selection".
+// Method: "Token Sparse Attention" papernotes.org notes, 关键设计 2 (each head keeps its
+// own top-k_keep tokens); gist.science §2 "Head-Wise Selection".
 #include "common.cuh"
 
 namespace tsa {
 
 constexpr int kSelThreads = 1024;
-
-// Fixed-point mass of one score: floor(v * 2^62), exact for v in [0, 1].
-__device__ inline unsigned long long mass62(uint32_t key) {
-    return __double2ull_rz((double)__uint_as_float(key) * 4611686018427387904.0);
-}
-
-// One block per batch element.  Finds k = min{k : sum of the k smallest masses >= T}
-// by refining an 8-bit digit of the key per pass, most significant first.
-__global__ void __launch_bounds__(kSelThreads)
-k_budget(const float *__restrict__ s_l, int L, unsigned long long T, int32_t *__restrict__ Lkeep,
-         Control *ctl) {
-    const int b = blockIdx.x;
-    const float *s = s_l + (size_t)b * L;
-    __shared__ unsigned int cnt[256];
-    __shared__ unsigned long long mass[256];
-    __shared__ uint32_t s_prefix, s_mask;
-    __shared__ unsigned long long s_before;
-    __shared__ int s_cbefore, s_done, s_k;
-    if (T == 0ull) {
-        if (threadIdx.x == 0) Lkeep[b] = L;
-        return;
-    }
-    if (threadIdx.x == 0) { s_prefix = 0; s_mask = 0; s_before = 0; s_cbefore = 0; s_done = 0; }
-    bool bad = false;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) { cnt[i] = 0; mass[i] = 0; }
-        __syncthreads();
-        const uint32_t prefix = s_prefix, mask = s_mask;
-        for (int t = threadIdx.x; t < L; t += blockDim.x) {
-            const uint32_t key = score_key<kLayerScoreMax>(s[t], bad);
-            if ((key & mask) == prefix) {
-                const int dg = (key >> shift) & 255;
-                atomicAdd(&cnt[dg], 1u);
-                const unsigned long long m = mass62(key);
-                if (m) atomicAdd(&mass[dg], m);
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            unsigned long long acc = s_before;
-            int c = s_cbefore, dg = -1;
-            for (int i = 0; i < 256; ++i) {
-                if (acc + mass[i] >= T) { dg = i; break; }
-                acc += mass[i];
-                c += cnt[i];
-            }
-            if (dg < 0) {  // total mass below the threshold: prune everything
-                s_done = 1;
-                s_k = L;
-            } else {
-                s_before = acc;
-                s_cbefore = c;
-                s_prefix = prefix | ((uint32_t)dg << shift);
-                s_mask = mask | (255u << shift);
-            }
-        }
-        __syncthreads();
-        if (s_done) break;
-    }
-    if (threadIdx.x == 0) {
-        int k = s_k;
-        if (!s_done) {
-            const unsigned long long a = mass62(s_prefix);  // > 0 by construction
-            const unsigned long long need = T - s_before;
-            k = s_cbefore + (int)((need + a - 1) / a);
-        }
-        Lkeep[b] = L - k;
-    }
-    if (bad) report_error(ctl, TSA_ERR_NONFINITE, 1);
-}
 
 // Exclusive block-wide prefix count of a 0/1 flag; returns the prefix, sets total.
 __device__ inline int block_scan_flag(bool f, int *warp_tot, int &total) {
@@ -171,13 +99,6 @@ k_select(const float *__restrict__ s_h, int L, int H, const int32_t *__restrict_
         base_eq += n_eq;
     }
     if (bad) report_error(ctl, TSA_ERR_NONFINITE, 3);
-}
-
-cudaError_t launch_budget(const tsa_dims &dm, const float *s_l, double tau, int32_t *Lkeep,
-                          Control *ctl, cudaStream_t st) {
-    const unsigned long long T = (unsigned long long)ceil(tau * 4611686018427387904.0);
-    k_budget<<<dm.B, kSelThreads, 0, st>>>(s_l, dm.L, T, Lkeep, ctl);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_select(const tsa_dims &dm, const float *s_h, const int32_t *Lkeep,
