@@ -1,20 +1,28 @@
 // Causal flash attention on the 5th-generation tensor cores (tcgen05 + TMEM), bf16 in,
 // fp32 accumulate, for the compressed L'×L' problem of each head and for the dense GQA
-// layer.  One CTA per 128-row query tile, heaviest (longest causal) tiles first.
+// layer.
 //
 // Method: "Token Sparse Attention" papernotes.org notes, 整体框架 (dense attention on the
 // compressed problem, complexity O(L'^2 d)); bxzpzcl.cn post §1.1 (softmax(Q̂K̂ᵀ/√d)V̂).
 // The causal mask j <= i in compressed order is the mask on original positions because
 // the index lists are ascending.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q tile once, then K and V tiles through a 2-stage ring.
-//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM S buffers,
-//               then O += P_j V_j with P_j read from TMEM (bf16, written over S_j).
-//   warps 4-7   softmax: thread r owns query row r.  Online max/sum in log2 units with a
-//               lazy O rescale (only when the running max grows by more than 2^8), P
-//               written back to TMEM, then the epilogue O / l -> bf16 -> global.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d).
+// One CTA per pair of 128-row query tiles (A = 2p, B = 2p+1) of one head; every K/V
+// tile is loaded once and used by both.  Pairs are scheduled heaviest first.
+// Warp roles (384 threads):
+//   warp 0      TMA producer: both Q tiles once, then K and V tiles through a 2-stage ring.
+//   warp 1      TMEM owner and MMA issuer.  Order per key tile j:
+//                 PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
+//               so that the softmax of one tile overlaps the MMAs of the other.  S = Q K^T
+//               goes to the tile's TMEM S buffer; O += P V reads P (bf16, written over S)
+//               from TMEM and V from shared memory.
+//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: thread r owns query row r.
+//               Online max/sum in log2 units; O is rescaled only when the running max grows
+//               by more than 2^8 (so P <= 2^8); P is written back to TMEM; the epilogue
+//               writes O / l as bf16.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+d), O_B [384, 384+d).
+// Because S_X(j+1) is issued after PV_X(j), its completion also means PV_X(j) is done:
+// the softmax may rescale O_X right after S_X(j+1) arrives.
 // Every wait is bounded in time; a wait that runs out records TSA_ERR_DEVICE_TIMEOUT,
 // the CTA drains its in-flight copies and MMAs, frees TMEM and exits.
 #include <math.h>
@@ -28,20 +36,104 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kStages = 2, kThreads = 256;
+constexpr int kBM = 128, kBN = 128, kStages = 2, kThreads = 384;
 constexpr uint64_t kDrainNs = 1000000000ull;  // drain waits: 1 s
 
 template <int D> struct AttnSmem {
     static constexpr int TILE = kBM * D * 2;  // bytes of a 128-row tile
-    alignas(1024) uint8_t q[TILE];
+    alignas(1024) uint8_t q[2][TILE];
     alignas(1024) uint8_t k[kStages][TILE];
     alignas(1024) uint8_t v[kStages][TILE];
     uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-    uint64_t s_full[2], p_full[2], pv_done, o_final, drain;
+    uint64_t s_full[2], p_full[2], o_final[2], drain;
     uint32_t tmem_base;
     int abort;
     int never;  // stays 0: drain waits ignore the abort flag
 };
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Softmax of one query tile (this warpgroup), steps j = 0..n-1; the last step is the
+// diagonal key tile.  Returns false if a wait ran out.
+template <int D>
+__device__ __forceinline__ bool softmax_tile(AttnSmem<D> &sm, int X, int n, uint32_t tS,
+                                             uint32_t tO, int r, uint32_t lo, float sl2,
+                                             uint64_t limit_ns, volatile int *abort, float &l_out) {
+    float m = -INFINITY, l = 0.0f;
+    for (int j = 0; j < n; ++j) {
+        bool ok = mbar_wait(&sm.s_full[X], j & 1, limit_ns, abort);
+        if (!__all_sync(0xffffffffu, ok)) return false;
+        tc_fence_after();
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            tmem_ld32(tS + lo + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld_wait();
+        if (j == n - 1) {  // diagonal tile: key c is visible to row r iff c <= r
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+                if (c > r) sr[c] = __float_as_uint(-INFINITY);
+        }
+        float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+#pragma unroll
+        for (int c = 2; c < 126; c += 4) {
+            mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+            mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+        }
+        const float mt =
+            fmax3(mx0, mx1, fmaxf(__uint_as_float(sr[126]), __uint_as_float(sr[127]))) * sl2;
+        float mu = m, factor = 1.0f;
+        bool resc = false;
+        if (m == -INFINITY) {
+            mu = mt;
+            factor = 0.0f;
+        } else if (mt > m + 8.0f) {
+            mu = mt;
+            factor = ex2(m - mt);
+            resc = true;
+        }
+        m = mu;
+        float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+            const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mu));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mu));
+            const float p2 = ex2(fmaf(__uint_as_float(sr[2 * c + 2]), sl2, -mu));
+            const float p3 = ex2(fmaf(__uint_as_float(sr[2 * c + 3]), sl2, -mu));
+            s0 += p0;
+            s1 += p1;
+            s2 += p2;
+            s3 += p3;
+            sr[c] = pack_bf16(p0, p1);  // in place: sr[c] and sr[c+1] were already read
+            sr[c + 1] = pack_bf16(p2, p3);
+        }
+        l = l * factor + ((s0 + s1) + (s2 + s3));
+        if (__any_sync(0xffffffffu, resc)) {
+            // S_X(j) was issued after PV_X(j-1), so O_X is complete here.
+            const float f = resc ? factor : 1.0f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + lo + c * 32, o);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                tmem_st32(tO + lo + c * 32, o);
+            }
+        }
+        tmem_st32(tS + lo, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_st32(tS + lo + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[X]);
+    }
+    l_out = l;
+    return true;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -53,14 +145,16 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     AttnSmem<D> &sm = *reinterpret_cast<AttnSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int TILE = AttnSmem<D>::TILE, NDB = D / 64;
-    const int ntiles = ceil_div(L, kBM);
-    const int BH = gridDim.x / ntiles;
-    const int tile = ntiles - 1 - (int)(blockIdx.x / BH), bh = blockIdx.x % BH;
+    const int npairs = ceil_div(L, 2 * kBM);
+    const int BH = gridDim.x / npairs;
+    const int pair = npairs - 1 - (int)(blockIdx.x / BH), bh = blockIdx.x % BH;
     const int b = bh / H, h = bh % H;
     const int Lk = dense ? L : __ldg(Lkeep + b);
-    const int i0 = tile * kBM;
+    const int i0 = pair * 2 * kBM;  // first row of tile A
     if (i0 >= Lk) return;
-    const int n_kv = tile + 1;
+    const bool hasB = i0 + kBM < Lk;
+    const int nA = 2 * pair + 1, nB = hasB ? 2 * pair + 2 : 0;
+    const int nkv = hasB ? nB : nA;
     const int kvh = dense ? h / (H / Hkv) : h;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -72,12 +166,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.v_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.s_full[i], 1);
-            mbar_init(&sm.p_full[i], 128);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&sm.s_full[x], 1);
+            mbar_init(&sm.p_full[x], 128);
+            mbar_init(&sm.o_final[x], 1);
         }
-        mbar_init(&sm.pv_done, 1);
-        mbar_init(&sm.o_final, 1);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         sm.never = 0;
@@ -91,18 +184,20 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
     volatile int *abort = &sm.abort;
     bool ok = true;
 
     if (warp == 0) {
         if (lane == 0) {
-            int issued = 0;  // K/V tiles issued
-            mbar_expect_tx(&sm.q_full, TILE);
+            int issued = 0;  // K/V tiles issued (negative: K of tile -issued-1 only)
+            mbar_expect_tx(&sm.q_full, 2 * TILE);
 #pragma unroll
-            for (int db = 0; db < NDB; ++db)
-                tma_load_4d(sm.q + db * kBM * 128, &tmQ, &sm.q_full, db * 64, i0, h, b);
-            for (int j = 0; j < n_kv; ++j) {
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int db = 0; db < NDB; ++db)
+                    tma_load_4d(sm.q[x] + db * kBM * 128, &tmQ, &sm.q_full, db * 64,
+                                i0 + x * kBM, h, b);
+            for (int j = 0; j < nkv; ++j) {
                 const int s = j % kStages;
                 const uint32_t ph = ((j / kStages) & 1) ^ 1;
                 if (!(ok = mbar_wait(&sm.k_empty[s], ph, limit_ns, abort))) break;
@@ -112,7 +207,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     tma_load_4d(sm.k[s] + db * kBN * 128, &tmK, &sm.k_full[s], db * 64, j * kBN,
                                 kvh, b);
                 if (!(ok = mbar_wait(&sm.v_empty[s], ph, limit_ns, abort))) {
-                    issued = -(j + 1);  // K_j in flight, V_j not issued
+                    issued = -(j + 1);
                     break;
                 }
                 mbar_expect_tx(&sm.v_full[s], TILE);
@@ -134,43 +229,53 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16(kBM, kBN, false);
             constexpr uint32_t idO = idesc_bf16(kBM, D, true);
-            const uint32_t qa = smem_u32(sm.q);
             bool any = false;
-            auto issue_S = [&](int j) -> bool {
-                const int s = j % kStages;
-                if (!mbar_wait(&sm.k_full[s], (j / kStages) & 1, limit_ns, abort)) return false;
-                tc_fence_after();
-                const uint32_t ka = smem_u32(sm.k[s]);
-                const uint32_t dS = (j & 1) ? tS1 : tS0;
+            auto S_mma = [&](int x, int j) {
+                const uint32_t qa = smem_u32(sm.q[x]), ka = smem_u32(sm.k[j % kStages]);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk / 4) * (kBM * 128) + (kk % 4) * 32;
-                    mma_ss(dS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                           idS, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + x * 128, sdesc_sw128(qa + off, 16, 1024),
+                           sdesc_sw128(ka + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
                 }
+                mma_commit(&sm.s_full[x]);
                 any = true;
-                mma_commit(&sm.k_empty[s]);
-                mma_commit(&sm.s_full[j & 1]);
-                return true;
             };
-            ok = mbar_wait(&sm.q_full, 0, limit_ns, abort);
-            if (ok) ok = issue_S(0);
-            if (ok && n_kv > 1) ok = issue_S(1);
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int s = j % kStages;
-                if (!(ok = mbar_wait(&sm.p_full[j & 1], (j >> 1) & 1, limit_ns, abort))) break;
-                if (!(ok = mbar_wait(&sm.v_full[s], (j / kStages) & 1, limit_ns, abort))) break;
-                tc_fence_after();
-                const uint32_t va = smem_u32(sm.v[s]);
-                const uint32_t aP = (j & 1) ? tS1 : tS0;
+            auto PV_mma = [&](int x, int j) {
+                const uint32_t va = smem_u32(sm.v[j % kStages]);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts(tO, aP + kk * 8, sdesc_sw128(va + kk * 2048, kBN * 128, 1024), idO,
+                    mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
+                           sdesc_sw128(va + kk * 2048, kBN * 128, 1024), idO,
                            (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&sm.v_empty[s]);
-                mma_commit(&sm.pv_done);
-                if (j == n_kv - 1) mma_commit(&sm.o_final);
-                if (j + 2 < n_kv) ok = issue_S(j + 2);
+            };
+            ok = mbar_wait(&sm.q_full, 0, limit_ns, abort) &&
+                 mbar_wait(&sm.k_full[0], 0, limit_ns, abort);
+            if (ok) {
+                tc_fence_after();
+                S_mma(0, 0);
+                if (hasB) S_mma(1, 0);
+                mma_commit(&sm.k_empty[0]);
+            }
+            for (int j = 0; j < nkv && ok; ++j) {
+                const bool next = j + 1 < nkv;
+                if (!(ok = mbar_wait(&sm.v_full[j % kStages], (j / kStages) & 1, limit_ns, abort)))
+                    break;
+                if (next && !(ok = mbar_wait(&sm.k_full[(j + 1) % kStages],
+                                             ((j + 1) / kStages) & 1, limit_ns, abort)))
+                    break;
+                for (int x = 0; x < 2; ++x) {
+                    const int nx = x ? nB : nA;
+                    if (j >= nx) continue;
+                    if (!(ok = mbar_wait(&sm.p_full[x], j & 1, limit_ns, abort))) break;
+                    tc_fence_after();
+                    PV_mma(x, j);
+                    if (j == nx - 1) mma_commit(&sm.o_final[x]);
+                    else S_mma(x, j + 1);
+                }
+                if (!ok) break;
+                mma_commit(&sm.v_empty[j % kStages]);
+                if (next) mma_commit(&sm.k_empty[(j + 1) % kStages]);
             }
             if (any) {  // every MMA issued here has completed before TMEM is freed
                 mma_commit(&sm.drain);
@@ -178,103 +283,46 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             }
         }
     } else if (warp >= 4) {
+        const int X = (warp - 4) >> 2;  // 0: tile A (warps 4-7), 1: tile B (warps 8-11)
         const int wq = warp & 3, r = wq * 32 + lane;
         const uint32_t lo = (uint32_t)(wq * 32) << 16;
-        float m = -INFINITY, l = 0.0f;
-        for (int j = 0; j < n_kv; ++j) {
-            ok = mbar_wait(&sm.s_full[j & 1], (j >> 1) & 1, limit_ns, abort);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t tS = ((j & 1) ? tS1 : tS0) + lo;
-            uint32_t sr[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-            tmem_ld_wait();
-            const bool diag = (j == n_kv - 1);
-            float mt = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                float v = __uint_as_float(sr[c]);
-                if (diag && c > r) v = -INFINITY;
-                sr[c] = __float_as_uint(v);
-                mt = fmaxf(mt, v);
-            }
-            mt *= sl2;
-            float mu = m, factor = 1.0f;
-            bool resc = false;
-            if (m == -INFINITY) {
-                mu = mt;
-                factor = 0.0f;
-            } else if (mt > m + 8.0f) {
-                mu = mt;
-                factor = ex2(m - mt);
-                resc = true;
-            }
-            m = mu;
-            float sum = 0.0f;
-            uint32_t pk[64];
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mu));
-                const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mu));
-                sum += p0 + p1;
-                pk[c] = pack_bf16(p0, p1);
-            }
-            l = l * factor + sum;
-            if (j > 0 && __any_sync(0xffffffffu, resc)) {
-                // PV_{j-2} is complete (S_j was issued after it and has completed), so the
-                // parity of phase j-1 identifies PV_{j-1} unambiguously.
-                ok = mbar_wait(&sm.pv_done, (j - 1) & 1, limit_ns, abort);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        const int n = X ? nB : nA;
+        if (n > 0) {
+            const uint32_t tS = tmem + X * 128, tO = tmem + 256 + X * 128;
+            float l = 1.0f;
+            ok = softmax_tile<D>(sm, X, n, tS, tO, r, lo, sl2, limit_ns, abort, l);
+            if (ok) ok = mbar_wait(&sm.o_final[X], 0, limit_ns, abort);
+            if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
-                const float f = resc ? factor : 1.0f;
+                const int i = i0 + X * kBM + r;
+                const float inv = 1.0f / l;
+                __nv_bfloat16 *orow = dense ? O + (((size_t)b * L + i) * H + h) * D
+                                            : O + ((size_t)bh * L + i) * D;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
                     tmem_ld32(tO + lo + c * 32, o);
                     tmem_ld_wait();
+                    if (i < Lk) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    tmem_st32(tO + lo + c * 32, o);
-                }
-                tmem_st_wait();
-            }
-            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&sm.p_full[j & 1]);
-        }
-        // O is final once the last O += P V has completed.  (A parity wait on pv_done
-        // cannot tell that phase from the one before it, which may still be pending.)
-        if (ok) ok = mbar_wait(&sm.o_final, 0, limit_ns, abort);
-        if (__all_sync(0xffffffffu, ok)) {
-            tc_fence_after();
-            const int i = i0 + r;
-            const float inv = 1.0f / l;
-            __nv_bfloat16 *orow = dense ? O + (((size_t)b * L + i) * H + h) * D
-                                        : O + ((size_t)bh * L + i) * D;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + lo + c * 32, o);
-                tmem_ld_wait();
-                if (i < Lk) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(o[q4 * 8 + 0]) * inv, __uint_as_float(o[q4 * 8 + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(o[q4 * 8 + 2]) * inv, __uint_as_float(o[q4 * 8 + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(o[q4 * 8 + 4]) * inv, __uint_as_float(o[q4 * 8 + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(o[q4 * 8 + 6]) * inv, __uint_as_float(o[q4 * 8 + 7]) * inv);
-                        dst[q4] = w;
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 w;
+                            w.x = pack_bf16(__uint_as_float(o[q4 * 8 + 0]) * inv,
+                                            __uint_as_float(o[q4 * 8 + 1]) * inv);
+                            w.y = pack_bf16(__uint_as_float(o[q4 * 8 + 2]) * inv,
+                                            __uint_as_float(o[q4 * 8 + 3]) * inv);
+                            w.z = pack_bf16(__uint_as_float(o[q4 * 8 + 4]) * inv,
+                                            __uint_as_float(o[q4 * 8 + 5]) * inv);
+                            w.w = pack_bf16(__uint_as_float(o[q4 * 8 + 6]) * inv,
+                                            __uint_as_float(o[q4 * 8 + 7]) * inv);
+                            dst[q4] = w;
+                        }
                     }
                 }
+            } else {
+                ok = false;
             }
-        } else {
-            ok = false;
         }
     }
     if (!ok) {
@@ -317,7 +365,7 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
     cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const long nblocks = (long)ceil_div(dm.L, kBM) * dm.B * dm.H;
+    const long nblocks = (long)ceil_div(dm.L, 2 * kBM) * dm.B * dm.H;
     k_attn_tc<D><<<(unsigned)nblocks, kThreads, smem, st>>>(
         tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
         (__nv_bfloat16 *)O, ctl, (uint64_t)limit_us * 1000ull);
