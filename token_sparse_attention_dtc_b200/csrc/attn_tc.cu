@@ -8,7 +8,7 @@
 // the index lists are ascending.
 //
 // One CTA per pair of 128-row query tiles (A = 2p, B = 2p+1) of one head; every K/V
-// tile is loaded once and used by both.  Pairs are scheduled heaviest first.
+// tile is loaded once and used by both.  CTAs run head by head, heaviest pairs first.
 // Warp roles (384 threads):
 //   warp 0      TMA producer: both Q tiles once, then K and V tiles through a 2-stage ring.
 //   warp 1      TMEM owner and MMA issuer.  Order per key tile j:
@@ -145,9 +145,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     AttnSmem<D> &sm = *reinterpret_cast<AttnSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int TILE = AttnSmem<D>::TILE, NDB = D / 64;
+    // Head-major order: the CTAs in flight together work on the same head (heaviest pairs
+    // first), so they walk the same K/V tiles at the same pace and share them in L2.
     const int npairs = ceil_div(L, 2 * kBM);
-    const int BH = gridDim.x / npairs;
-    const int pair = npairs - 1 - (int)(blockIdx.x / BH), bh = blockIdx.x % BH;
+    const int bh = blockIdx.x / npairs, pair = npairs - 1 - (int)(blockIdx.x % npairs);
     const int b = bh / H, h = bh % H;
     const int Lk = dense ? L : __ldg(Lkeep + b);
     const int i0 = pair * 2 * kBM;  // first row of tile A
