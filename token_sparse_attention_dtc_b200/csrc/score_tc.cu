@@ -18,7 +18,9 @@
 //   s_h[b, h, t].  The CTA walks its token range backwards, so its first tiles are the
 //   ones pass 1 read last (likely still in L2).
 // Both passes: warp 0 streams K tiles by TMA through a 4-stage ring, warp 1 issues the
-// MMAs into two TMEM accumulators, warps 4-7 run the epilogue.  All waits are bounded.
+// MMAs into two TMEM accumulators, warps 4-19 run the epilogue (4 TMEM lane quadrants x
+// 4 column groups, so each thread handles a quarter of a tile's columns).  All waits are
+// bounded.
 #include <math.h>
 
 #include <algorithm>
@@ -30,7 +32,8 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 256, kStages = 4, kTile = 128;
+constexpr int kThreads = 640, kStages = 4, kTile = 128;
+constexpr int kEpiWarps = 16;  // warps 4..19: 4 TMEM lane quadrants x 4 column groups
 constexpr uint64_t kDrainNs = 1000000000ull;
 
 template <int D> struct ScoreSmem {
@@ -38,7 +41,8 @@ template <int D> struct ScoreSmem {
     alignas(1024) uint8_t q[2 * 128 * D * 2];  // up to 256 query rows, swizzled, K-major
     alignas(1024) uint8_t k[kStages][KT];
     uint64_t k_full[kStages], k_empty[kStages], acc_full[2], acc_empty[2], drain;
-    float2 stat[256];  // pass 2: (max, 1/sum) per query row
+    float2 stat[256];          // pass 2: (max, 1/sum) per query row
+    float2 red[4][256];        // pass 1: per column group (max, sum) per query row
     uint32_t tmem_base;
     int abort, never;
 };
@@ -97,7 +101,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sm.acc_full[a], 1);
-            mbar_init(&sm.acc_empty[a], 128);
+            mbar_init(&sm.acc_empty[a], kEpiWarps * 32);
         }
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
@@ -181,11 +185,14 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
             }
         }
     } else if (warp >= 4) {
-        const int wq = warp & 3, r = wq * 32 + lane;
+        // Epilogue warp (wq, cg): TMEM lane quadrant wq = warp % 4 (the lanes this warp may
+        // read), column group cg = (warp - 4) / 4.
+        const int wq = warp & 3, cg = (warp - 4) >> 2, r = wq * 32 + lane;
         const uint32_t lo = (uint32_t)(wq * 32) << 16;
         const int pmin = L - qe;  // first recent-query position
         if (!kPass2) {
-            // thread r owns query rows r (+128 for a second row block)
+            // Thread owns query row r (+128 in a second row block) over the tile columns
+            // [cg*32, cg*32 + 32); the four column groups are merged at the end.
             float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
             int pr[2];
             for (int rb = 0; rb < 2; ++rb) {
@@ -197,73 +204,83 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                 ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
-                const int t0 = tile_at(it) * kTile;
-                const bool tail = t0 + kTile - 1 > pmin;  // some token may follow a query
+                const int tc0 = tile_at(it) * kTile + cg * 32;  // token of column 0 here
+                const bool tail = tc0 + 31 > pmin;  // some token may follow a query
                 for (int rb = 0; rb < RB; ++rb) {
                     if (rb * 128 + wq * 32 >= N) continue;  // whole warp on padding rows
+                    uint32_t v[32];
+                    tmem_ld32(tmem + a * acc_cols + rb * 128 + cg * 32 + lo, v);
+                    tmem_ld_wait();
+                    if (pr[rb] < 0) continue;
+                    float cm = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < kTile / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + a * acc_cols + rb * 128 + c * 32 + lo, v);
-                        tmem_ld_wait();
-                        if (pr[rb] < 0) continue;
-                        float cm = -INFINITY;
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            float z = __uint_as_float(v[e]);
-                            if (tail && t0 + c * 32 + e > pr[rb]) z = -INFINITY;
-                            v[e] = __float_as_uint(z);
-                            cm = fmaxf(cm, z);
-                        }
-                        if (cm == -INFINITY) continue;
-                        cm *= sl2;
-                        if (cm > m[rb]) {
-                            l[rb] = (m[rb] == -INFINITY) ? 0.0f : l[rb] * ex2(m[rb] - cm);
-                            m[rb] = cm;
-                        }
-                        float acc = 0.0f;
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            acc += ex2(fmaf(__uint_as_float(v[e]), sl2, -m[rb]));
-                        l[rb] += acc;
+                    for (int e = 0; e < 32; ++e) {
+                        float z = __uint_as_float(v[e]);
+                        if (tail && tc0 + e > pr[rb]) z = -INFINITY;
+                        v[e] = __float_as_uint(z);
+                        cm = fmaxf(cm, z);
                     }
+                    if (cm == -INFINITY) continue;
+                    cm *= sl2;
+                    if (cm > m[rb]) {
+                        l[rb] = (m[rb] == -INFINITY) ? 0.0f : l[rb] * ex2(m[rb] - cm);
+                        m[rb] = cm;
+                    }
+                    float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        a0 += ex2(fmaf(__uint_as_float(v[e]), sl2, -m[rb]));
+                        a1 += ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -m[rb]));
+                    }
+                    l[rb] += a0 + a1;
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.acc_empty[a]);
             }
-            if (ok)
+            for (int rb = 0; rb < RB; ++rb) sm.red[cg][rb * 128 + r] = make_float2(m[rb], l[rb]);
+            named_barrier(1, kEpiWarps * 32);
+            ok = __all_sync(0xffffffffu, ok) && !*abort;
+            if (ok && cg == 0)
                 for (int rb = 0; rb < RB; ++rb) {
                     const int n = rb * 128 + r;
-                    if (n < N) part[((size_t)bg * nsplit + split) * N + n] = make_float2(m[rb], l[rb]);
+                    if (n >= N) continue;
+                    float mm = -INFINITY, ll = 0.0f;
+                    for (int g2 = 0; g2 < 4; ++g2) {  // fixed merge order
+                        const float2 p = sm.red[g2][n];
+                        const float mx = fmaxf(mm, p.x);
+                        const float x = (mm == -INFINITY) ? 0.0f : ll * ex2(mm - mx);
+                        const float y = (p.x == -INFINITY) ? 0.0f : p.y * ex2(p.x - mx);
+                        mm = mx;
+                        ll = x + y;
+                    }
+                    part[((size_t)bg * nsplit + split) * N + n] = make_float2(mm, ll);
                 }
         } else {
-            const int nchunks = Npad / 32 + ((Npad % 32) ? 1 : 0);
+            // Thread owns token r of the tile and the heads g = cg, cg + 4, ...; head g's
+            // query rows are the columns [g*qe, (g+1)*qe), summed in row order.
             for (int it = 0; it < count; ++it) {
                 const int a = it & 1;
                 ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
                 const int t = tile_at(it) * kTile + r;
-                int g = 0, i = 0;
-                float acc = 0.0f;
-                for (int c = 0; c < nchunks; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + a * acc_cols + c * 32 + lo, v);
-                    tmem_ld_wait();
+                for (int g = cg; g < G; g += 4) {
+                    const int c0 = g * qe, c1 = c0 + qe;
+                    float acc = 0.0f;
+                    for (int cs = c0 & ~15; cs < c1; cs += 16) {
+                        uint32_t v[16];
+                        tmem_ld16(tmem + a * acc_cols + cs + lo, v);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int n = c * 32 + e;
-                        if (n >= N) break;
-                        const float2 st = sm.stat[n];
-                        if (t <= pmin + i)
-                            acc = fmaf(ex2(fmaf(__uint_as_float(v[e]), sl2, -st.x)), st.y, acc);
-                        if (++i == qe) {
-                            if (t < L) s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
-                            acc = 0.0f;
-                            i = 0;
-                            ++g;
+                        for (int e = 0; e < 16; ++e) {
+                            const int n = cs + e;
+                            if (n < c0 || n >= c1) continue;
+                            const float2 st = sm.stat[n];
+                            if (t <= pmin + (n - c0))
+                                acc = fmaf(ex2(fmaf(__uint_as_float(v[e]), sl2, -st.x)), st.y, acc);
                         }
                     }
+                    if (t < L) s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.acc_empty[a]);
