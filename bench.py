@@ -57,6 +57,23 @@ def _traffic(kernel: str, workload: str):
     return e["bytes_per_launch"] if h == e["source_sha"] else None
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own sequence (batch sharding)."""
+    return seed * 1000 + rank
+
+
+def job_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank value over all ranks (the job's time); identity on one rank."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
 
@@ -197,7 +214,7 @@ def run_ours(args, w, L, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     tsa.lib()  # fail loudly if the CUDA library is missing
-    x = make_workload(w.name, seed=args.seed * 1000 + rank, L=L, B=1)
+    x = make_workload(w.name, seed=rank_seed(args.seed, rank), L=L, B=1)
     d = {k: v.to(dev) for k, v in x.items()}
     dm = tsa.dims(d["Q"], d["K"])
     ws = tsa.workspace(dm, w.q, layer=True, device=dev)
@@ -240,10 +257,7 @@ def run_ours(args, w, L, rank, world, local_rank):
     lk = int(Lk.item())
     if tsa.tsa_get_device_status(ws) != 0:
         raise RuntimeError("device error during the timed region")
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = job_max(ms_step, world, dev)
 
     peaks = _peaks()
     flops = 2.0 * w.H * w.d * lk * (lk + 1)
@@ -317,11 +331,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             e2e_step()
         b.record(st)
         sync_all()
-        ems = a.elapsed_time(b) / ne
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = job_max(a.elapsed_time(b) / ne, world, dev)
         e2e = {"value": ems / world, "unit": "ms", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": ne}
 

@@ -195,6 +195,13 @@ TSA_API tsa_status tsa_get_device_status(void *ws, void *stream);
  * tensor memory and exit; tests lower the limit to check that path. */
 TSA_API void tsa_set_wait_limit(uint32_t microseconds);
 
+/* Test hook for the failure path, off by default.  When `on` is non-zero, later launches
+ * of the tensor-core kernels (scoring of bf16 inputs, attention of bf16 inputs) first
+ * make their MMA-issuing thread wait on a barrier that nothing completes.  The wait
+ * runs out after the wait limit; the kernel then records TSA_ERR_DEVICE_TIMEOUT, winds
+ * down as described above, and exits.  Nothing faults, traps or hangs. */
+TSA_API void tsa_set_test_stall(int32_t on);
+
 TSA_API const char *tsa_status_string(tsa_status s);
 TSA_API const char *tsa_last_error(void);
 

@@ -1,0 +1,94 @@
+"""Failure detection on the GPU, without faulting it.
+
+Every device-side wait in the tensor-core kernels is bounded in time.  The test hook
+tsa_set_test_stall makes each kernel's MMA issuer wait on a barrier that nothing
+completes; with a 20 ms limit that wait runs out, and the kernel must record
+TSA_ERR_DEVICE_TIMEOUT in the workspace, finish the copies and MMAs it started, free its
+tensor memory and exit.  The host reads the status, and the same context must then run
+the next launch correctly.
+"""
+import pytest
+import torch
+
+from token_sparse_attention_dtc_b200 import tsa
+from token_sparse_attention_dtc_b200.inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+DEFAULT_LIMIT_US = 2_000_000
+TIMEOUT = 6
+
+
+class stalled:
+    """Context: the test hook on, with a 20 ms wait limit."""
+
+    def __enter__(self):
+        tsa.tsa_set_wait_limit(20_000)
+        tsa.tsa_set_test_stall(True)
+
+    def __exit__(self, *a):
+        tsa.tsa_set_test_stall(False)
+        tsa.tsa_set_wait_limit(DEFAULT_LIMIT_US)
+
+
+def _stage_inputs():
+    x = make_inputs(1, 1000, 8, 2, 128, torch.bfloat16, seed=31)
+    d = {k: v.cuda() for k, v in x.items()}
+    dm = tsa.dims(d["Q"], d["K"])
+    ws = tsa.workspace(dm, 16)
+    s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
+    Lk = tsa.tsa_budget(dm, s_l, 0.02, ws=ws)
+    idx = tsa.tsa_select(dm, s_h, Lk, ws=ws)
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk)
+    assert tsa.tsa_get_device_status(ws) == 0
+    return d, dm, Lk, Qh, Kh, Vh, s_h, s_l
+
+
+def test_attention_wait_timeout_is_reported_and_context_recovers():
+    d, dm, Lk, Qh, Kh, Vh, _, _ = _stage_inputs()
+    lk = int(Lk.item())
+    ref = tsa.tsa_attn(dm, Qh, Kh, Vh, Lk)[:, :, :lk].clone()
+    ws = tsa.workspace(dm, 16)
+    with stalled():
+        tsa.tsa_attn(dm, Qh, Kh, Vh, Lk, ws=ws)
+        st = tsa.tsa_get_device_status(ws)
+    assert st == TIMEOUT
+    assert tsa.tsa_get_device_status(ws) == 0  # reading the status clears it
+    again = tsa.tsa_attn(dm, Qh, Kh, Vh, Lk, ws=ws)[:, :, :lk]
+    assert tsa.tsa_get_device_status(ws) == 0
+    assert torch.equal(again, ref)
+    # the dense mode goes through the same waits
+    with stalled():
+        tsa.tsa_attn(dm, d["Q"], d["K"], d["V"], None, dense=True, ws=ws)
+        st = tsa.tsa_get_device_status(ws)
+    assert st == TIMEOUT
+
+
+def test_scoring_wait_timeout_is_reported_and_context_recovers():
+    d, dm, _, _, _, _, s_h_ref, s_l_ref = _stage_inputs()
+    ws = tsa.workspace(dm, 16)
+    with stalled():
+        tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
+        st = tsa.tsa_get_device_status(ws)
+    assert st == TIMEOUT
+    s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
+    assert tsa.tsa_get_device_status(ws) == 0
+    assert torch.equal(s_h, s_h_ref) and torch.equal(s_l, s_l_ref)
+
+
+def test_out_of_range_scores_are_flagged():
+    """The budget and selection flag scores outside their legal range (NaN, < 0, or a
+    layer score above 1) instead of using them silently."""
+    dm = tsa.Dims(1, 4096, 2, 1, 64, tsa.TSA_BF16)
+    ws = tsa.workspace(dm, 1)
+    s = torch.full((1, 4096), 1.0 / 4096, device="cuda")
+    s[0, 17] = float("nan")
+    tsa.tsa_budget(dm, s, 0.01, ws=ws)
+    assert tsa.tsa_get_device_status(ws) == 7
+    sh = torch.rand(1, 2, 4096, device="cuda")
+    sh[0, 1, 5] = -1.0
+    tsa.tsa_select(dm, sh, torch.tensor([100], dtype=torch.int32, device="cuda"), ws=ws)
+    assert tsa.tsa_get_device_status(ws) == 7
+    # in-range scores give no error
+    tsa.tsa_budget(dm, torch.full((1, 4096), 1.0 / 4096, device="cuda"), 0.01, ws=ws)
+    assert tsa.tsa_get_device_status(ws) == 0

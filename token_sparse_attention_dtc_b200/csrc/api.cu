@@ -34,6 +34,9 @@ cudaError_t launch_scatter(const tsa_dims &, const void *, const int32_t *, cons
 
 static thread_local std::string g_last_error;
 static uint32_t g_wait_limit_us = 2000000;  // 2 s
+static int g_test_stall = 0;
+
+int test_stall() { return g_test_stall; }
 
 static tsa_status fail(tsa_status s, const char *fmt, ...) {
     char buf[512];
@@ -341,6 +344,8 @@ tsa_status tsa_get_device_status(void *ws, void *stream) {
 }
 
 void tsa_set_wait_limit(uint32_t microseconds) { g_wait_limit_us = microseconds; }
+
+void tsa_set_test_stall(int32_t on) { g_test_stall = on ? 1 : 0; }
 
 const char *tsa_status_string(tsa_status s) {
     switch (s) {

@@ -46,6 +46,7 @@ template <int D> struct AttnSmem {
     alignas(1024) uint8_t v[kStages][TILE];
     uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], o_final[2], drain;
+    uint64_t stall;  // test hook: initialised, never completed
     uint32_t tmem_base;
     int abort;
     int never;  // stays 0: drain waits ignore the abort flag
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ Lkeep, int dense,
           int L, int H, int Hkv, float sl2, __nv_bfloat16 *__restrict__ O, Control *ctl,
-          uint64_t limit_ns) {
+          uint64_t limit_ns, int stall) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem<D> &sm = *reinterpret_cast<AttnSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,6 +174,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             mbar_init(&sm.o_final[x], 1);
         }
         mbar_init(&sm.drain, 1);
+        mbar_init(&sm.stall, 1);
         sm.abort = 0;
         sm.never = 0;
         fence_mbar_init();
@@ -250,7 +252,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                            sdesc_sw128(va + kk * 2048, kBN * 128, 1024), idO,
                            (j > 0 || kk > 0) ? 1u : 0u);
             };
-            ok = mbar_wait(&sm.q_full, 0, limit_ns, abort) &&
+            // Test hook: a wait that nothing completes, so it runs out after limit_ns.
+            if (stall) ok = mbar_wait(&sm.stall, 0, limit_ns, abort);
+            ok = ok && mbar_wait(&sm.q_full, 0, limit_ns, abort) &&
                  mbar_wait(&sm.k_full[0], 0, limit_ns, abort);
             if (ok) {
                 tc_fence_after();
@@ -369,7 +373,7 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
     const long nblocks = (long)ceil_div(dm.L, 2 * kBM) * dm.B * dm.H;
     k_attn_tc<D><<<(unsigned)nblocks, kThreads, smem, st>>>(
         tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
-        (__nv_bfloat16 *)O, ctl, (uint64_t)limit_us * 1000ull);
+        (__nv_bfloat16 *)O, ctl, (uint64_t)limit_us * 1000ull, test_stall());
     return cudaGetLastError();
 }
 

@@ -87,4 +87,7 @@ struct WsLayout {
 
 WsLayout ws_layout(const tsa_dims &dm, int q);
 
+// Host: the failure-path test hook set by tsa_set_test_stall (0 or 1).
+int test_stall();
+
 }  // namespace tsa

@@ -41,6 +41,7 @@ template <int D> struct ScoreSmem {
     alignas(1024) uint8_t q[2 * 128 * D * 2];  // up to 256 query rows, swizzled, K-major
     alignas(1024) uint8_t k[kStages][KT];
     uint64_t k_full[kStages], k_empty[kStages], acc_full[2], acc_empty[2], drain;
+    uint64_t stall;  // test hook: initialised, never completed
     float2 stat[256];          // pass 2: (max, 1/sum) per query row
     float2 red[4][256];        // pass 1: per column group (max, sum) per query row
     uint32_t tmem_base;
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restrict__ Q, int L,
            int H, int Hkv, int qe, float sl2, int nsplit, float2 *__restrict__ part,
            const float2 *__restrict__ stat, float *__restrict__ s_h, Control *ctl,
-           uint64_t limit_ns) {
+           uint64_t limit_ns, int stall) {
     extern __shared__ uint8_t smem_raw[];
     ScoreSmem<D> &sm = *reinterpret_cast<ScoreSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -104,6 +105,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
             mbar_init(&sm.acc_empty[a], kEpiWarps * 32);
         }
         mbar_init(&sm.drain, 1);
+        mbar_init(&sm.stall, 1);
         sm.abort = 0;
         sm.never = 0;
         fence_mbar_init();
@@ -149,7 +151,9 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
             const uint32_t id1 = idesc_bf16(128, kTile, false);
             const uint32_t id2 = idesc_bf16(128, Npad, false);
             bool any = false;
-            for (int it = 0; it < count; ++it) {
+            // Test hook: a wait that nothing completes, so it runs out after limit_ns.
+            if (stall) ok = mbar_wait(&sm.stall, 0, limit_ns, abort);
+            for (int it = 0; it < count && ok; ++it) {
                 const int s = it % kStages, a = it & 1;
                 if (!(ok = mbar_wait(&sm.k_full[s], (it / kStages) & 1, limit_ns, abort))) break;
                 if (!(ok = mbar_wait(&sm.acc_empty[a], ((it >> 1) & 1) ^ 1, limit_ns, abort)))
@@ -349,13 +353,13 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
     dim3 grid(nsplit, dm.B * dm.Hkv);
     k_score_tc<D, false><<<grid, kThreads, smem, st>>>(tk, (const __nv_bfloat16 *)Q, dm.L, dm.H,
                                                        dm.Hkv, qe, sl2, nsplit, part, stat,
-                                                       s_h, ctl, lim);
+                                                       s_h, ctl, lim, test_stall());
     if ((e = cudaGetLastError())) return e;
     const int N = (dm.H / dm.Hkv) * qe;
     if ((e = launch_combine(part, nsplit, N, stat, dm.B * dm.Hkv, st))) return e;
     k_score_tc<D, true><<<grid, kThreads, smem, st>>>(tk, (const __nv_bfloat16 *)Q, dm.L, dm.H,
                                                       dm.Hkv, qe, sl2, nsplit, part, stat,
-                                                      s_h, ctl, lim);
+                                                      s_h, ctl, lim, test_stall());
     return cudaGetLastError();
 }
 

@@ -23,7 +23,7 @@ STATUS = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_ALIGNMENT",
 EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_budget",
            "tsa_select", "tsa_gather_qkv", "tsa_attn", "tsa_scatter_residual", "tsa_layer",
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
-           "tsa_last_error", "tsa_score_fixed_scratch")
+           "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall")
 
 
 class TSAError(RuntimeError):
@@ -59,6 +59,7 @@ def lib():
             "tsa_layer": (I32, [DP, P, P, P, P, P, I32, I32, D, F, P, P, P, P, P, SZ, P, P]),
             "tsa_get_device_status": (I32, [P, P]),
             "tsa_set_wait_limit": (None, [ctypes.c_uint32]),
+            "tsa_set_test_stall": (None, [I32]),
             "tsa_status_string": (ctypes.c_char_p, [I32]),
             "tsa_last_error": (ctypes.c_char_p, []),
             "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
@@ -233,5 +234,10 @@ def tsa_get_device_status(ws, stream=None) -> int:
     return int(st)
 
 
-def tsa_set_wait_limit(iterations: int):
-    lib().tsa_set_wait_limit(int(iterations))
+def tsa_set_wait_limit(microseconds: int):
+    lib().tsa_set_wait_limit(int(microseconds))
+
+
+def tsa_set_test_stall(on: bool):
+    """Failure-path test hook (see include/tsa.h)."""
+    lib().tsa_set_test_stall(1 if on else 0)
