@@ -1,4 +1,5 @@
-// Dynamic Token Coverage scoring on the tensor cores (bf16 inputs), exact two-pass softmax.
+// Dynamic Token Coverage scoring on the tensor cores (bf16 inputs), exact two-pass softmax
+// in one cooperative kernel.
 //
 // Method: "Token Sparse Attention" papernotes.org notes, 关键设计 2 (the last q queries
 // score all keys with a per-head softmax; column sums give s_h); bxzpzcl.cn post §2.1;
@@ -7,20 +8,23 @@
 // K tiles.  All logits are z2 = scale*log2(e)*<q, k> in fp32 (bf16 products, fp32
 // accumulation in TMEM).
 //
-// Pass 1 (k_score_stats_tc): S = Qblk · Ktile^T with the query rows on the TMEM lanes
-//   (M = 128 query rows, zero-padded; two row blocks when N > 128), 128 tokens per MMA.
-//   Each epilogue thread owns one query row and keeps its running (max, sum of 2^(z2-max))
-//   over the CTA's contiguous token range, so no cross-thread reduction is needed; the
-//   CTA writes one (max, sum) per row.  k_score_combine (score_simt.cu) merges the splits.
-// Pass 2 (k_score_colsum_tc): S^T = Ktile · Qblk^T with the tokens on the TMEM lanes
-//   (M = 128 tokens, N = query rows padded to 16).  Each thread owns one token and adds
-//   2^(z2 - max_n) / sum_n over the rows n of each head in row order, then stores
-//   s_h[b, h, t].  The CTA walks its token range backwards, so its first tiles are the
-//   ones pass 1 read last (likely still in L2).
-// Both passes: warp 0 streams K tiles by TMA through a 4-stage ring, warp 1 issues the
-// MMAs into two TMEM accumulators, warps 4-19 run the epilogue (4 TMEM lane quadrants x
-// 4 column groups, so each thread handles a quarter of a tile's columns).  All waits are
-// bounded.
+// Each CTA owns a contiguous range of K tiles of one group and walks it twice:
+// Pass 1 (ascending): S = Qblk · Ktile^T with the query rows on the TMEM lanes (M = 128
+//   query rows, zero-padded; two row blocks when N > 128).  Each epilogue thread keeps a
+//   running (max, sum of 2^(z2-max)) of one query row over a quarter of each tile's
+//   columns; the quarters are merged in a fixed order and the CTA writes one (max, sum)
+//   per row.
+// Grid barrier: the epilogue waits until every CTA has written its pass-1 pairs, then
+//   merges the pairs of its group in split order into (max, 1/sum) per row.  The
+//   producer and MMA warps do not wait: pass-2 MMAs need no statistics.
+// Pass 2 (descending, so the first tiles are the ones pass 1 read last and are likely
+//   still in L2): S^T = Ktile · Qblk^T with the tokens on the TMEM lanes (N = query rows
+//   padded to 16).  Each thread owns one token and adds 2^(z2 - max_n) / sum_n over the
+//   rows of the heads of its column group in row order, then stores s_h[b, h, t].
+// Warp 0 streams K tiles by TMA through a 4-stage ring, warp 1 issues the MMAs into two
+// TMEM accumulators, warps 4-19 run the epilogue (4 TMEM lane quadrants x 4 column
+// groups).  The grid is at most one CTA per SM and is launched cooperatively, so every
+// CTA is resident for the grid barrier.  All waits are bounded.
 #include <math.h>
 
 #include <algorithm>
@@ -41,11 +45,11 @@ template <int D> struct ScoreSmem {
     alignas(1024) uint8_t q[2 * 128 * D * 2];  // up to 256 query rows, swizzled, K-major
     alignas(1024) uint8_t k[kStages][KT];
     uint64_t k_full[kStages], k_empty[kStages], acc_full[2], acc_empty[2], drain;
-    uint64_t stall;  // test hook: initialised, never completed
-    float2 stat[256];          // pass 2: (max, 1/sum) per query row
-    float2 red[4][256];        // pass 1: per column group (max, sum) per query row
+    uint64_t stall;     // test hook: initialised, never completed
+    float2 stat[256];   // pass 2: (max, 1/sum) per query row
+    float2 red[4][256]; // pass 1: per column group (max, sum) per query row
     uint32_t tmem_base;
-    int abort, never;
+    int abort, never, gbar_ok;
 };
 
 // Copy the N recent-query rows of group (b, kv) into shared memory in the 128-byte swizzled
@@ -75,24 +79,34 @@ __device__ inline void tile_range(int ntiles, int nsplit, int split, int &first,
     count = per + (split < rem ? 1 : 0);
 }
 
-template <int D, bool kPass2>
+__device__ inline void online_merge(float &m, float &l, float m2, float l2) {
+    const float mx = fmaxf(m, m2);
+    const float a = (m == -INFINITY) ? 0.0f : l * ex2(m - mx);
+    const float c = (m2 == -INFINITY) ? 0.0f : l2 * ex2(m2 - mx);
+    m = mx;
+    l = a + c;
+}
+
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restrict__ Q, int L,
-           int H, int Hkv, int qe, float sl2, int nsplit, float2 *__restrict__ part,
-           const float2 *__restrict__ stat, float *__restrict__ s_h, Control *ctl,
-           uint64_t limit_ns, int stall) {
+           int H, int Hkv, int qe, float sl2, int nsplit, int group0, float2 *part,
+           float *__restrict__ s_h, unsigned int *gbar, Control *ctl, uint64_t limit_ns,
+           int stall) {
     extern __shared__ uint8_t smem_raw[];
     ScoreSmem<D> &sm = *reinterpret_cast<ScoreSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int KT = ScoreSmem<D>::KT, NDB = D / 64;
-    const int split = blockIdx.x, bg = blockIdx.y;
+    const int split = blockIdx.x, bg = group0 + blockIdx.y;
     const int b = bg / Hkv, kv = bg % Hkv, G = H / Hkv, N = G * qe;
-    const int RB = (N + 127) / 128;              // pass 1 row blocks
-    const int Npad = (N + 15) & ~15;             // pass 2 MMA N
-    const int nrows = kPass2 ? Npad : RB * 128;  // query rows held in shared memory
+    const int RB = (N + 127) / 128;   // pass 1 row blocks
+    const int Npad = (N + 15) & ~15;  // pass 2 MMA N
+    const int nrows = RB * 128;       // query rows held in shared memory
     const int ntiles = (L + kTile - 1) / kTile;
     int first, count;
     tile_range(ntiles, nsplit, split, first, count);
+    const int total = 2 * count;  // iterations over both passes
+    const unsigned nctas = gridDim.x * gridDim.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -108,11 +122,10 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
         mbar_init(&sm.stall, 1);
         sm.abort = 0;
         sm.never = 0;
+        sm.gbar_ok = 0;
         fence_mbar_init();
     }
     load_q_block<D>(sm.q, Q, b, kv, L, H, G, qe, N, nrows);
-    if (kPass2)
-        for (int n = threadIdx.x; n < N; n += kThreads) sm.stat[n] = stat[(size_t)bg * N + n];
     fence_proxy_async_smem();  // make the generic-proxy Q writes visible to the MMA
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, 512);
@@ -122,16 +135,15 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t acc_cols = kPass2 ? 256u : (uint32_t)RB * 128u;  // per accumulator
     volatile int *abort = &sm.abort;
     bool ok = true;
-    // Order of tiles: pass 1 ascending, pass 2 descending within the CTA's range.
-    auto tile_at = [&](int it) { return kPass2 ? first + count - 1 - it : first + it; };
+    // Tile of iteration it: pass 1 ascending, pass 2 descending within the CTA's range.
+    auto tile_at = [&](int it) { return it < count ? first + it : first + total - 1 - it; };
 
     if (warp == 0) {
         if (lane == 0) {
             int issued = 0;
-            for (int it = 0; it < count; ++it) {
+            for (int it = 0; it < total; ++it) {
                 const int s = it % kStages;
                 if (!(ok = mbar_wait(&sm.k_empty[s], ((it / kStages) & 1) ^ 1, limit_ns, abort)))
                     break;
@@ -153,20 +165,21 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
             bool any = false;
             // Test hook: a wait that nothing completes, so it runs out after limit_ns.
             if (stall) ok = mbar_wait(&sm.stall, 0, limit_ns, abort);
-            for (int it = 0; it < count && ok; ++it) {
+            for (int it = 0; it < total && ok; ++it) {
                 const int s = it % kStages, a = it & 1;
                 if (!(ok = mbar_wait(&sm.k_full[s], (it / kStages) & 1, limit_ns, abort))) break;
                 if (!(ok = mbar_wait(&sm.acc_empty[a], ((it >> 1) & 1) ^ 1, limit_ns, abort)))
                     break;
                 tc_fence_after();
                 const uint32_t ka = smem_u32(sm.k[s]);
-                const uint32_t dacc = tmem + a * acc_cols;
-                if (!kPass2) {
+                const uint32_t dacc = tmem + a * 256;
+                if (it < count) {
                     for (int rb = 0; rb < RB; ++rb)
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t kof = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
-                            const uint32_t qof = (kk / 4) * (nrows * 128) + rb * 128 * 128 + (kk % 4) * 32;
+                            const uint32_t qof =
+                                (kk / 4) * (nrows * 128) + rb * 128 * 128 + (kk % 4) * 32;
                             mma_ss(dacc + rb * 128, sdesc_sw128(qa + qof, 16, 1024),
                                    sdesc_sw128(ka + kof, 16, 1024), id1, kk > 0 ? 1u : 0u);
                         }
@@ -193,10 +206,10 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
         // read), column group cg = (warp - 4) / 4.
         const int wq = warp & 3, cg = (warp - 4) >> 2, r = wq * 32 + lane;
         const uint32_t lo = (uint32_t)(wq * 32) << 16;
-        const int pmin = L - qe;  // first recent-query position
-        if (!kPass2) {
-            // Thread owns query row r (+128 in a second row block) over the tile columns
-            // [cg*32, cg*32 + 32); the four column groups are merged at the end.
+        const int pmin = L - qe;           // first recent-query position
+        const int et = threadIdx.x - 128;  // 0..511 among the epilogue threads
+        // ---- pass 1: thread owns query row r (+128) over tile columns [cg*32, cg*32+32)
+        {
             float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.0f, 0.0f};
             int pr[2];
             for (int rb = 0; rb < 2; ++rb) {
@@ -213,7 +226,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                 for (int rb = 0; rb < RB; ++rb) {
                     if (rb * 128 + wq * 32 >= N) continue;  // whole warp on padding rows
                     uint32_t v[32];
-                    tmem_ld32(tmem + a * acc_cols + rb * 128 + cg * 32 + lo, v);
+                    tmem_ld32(tmem + a * 256 + rb * 128 + cg * 32 + lo, v);
                     tmem_ld_wait();
                     if (pr[rb] < 0) continue;
                     float cm = -INFINITY;
@@ -242,58 +255,81 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                 mbar_arrive(&sm.acc_empty[a]);
             }
             for (int rb = 0; rb < RB; ++rb) sm.red[cg][rb * 128 + r] = make_float2(m[rb], l[rb]);
-            named_barrier(1, kEpiWarps * 32);
-            ok = __all_sync(0xffffffffu, ok) && !*abort;
-            if (ok && cg == 0)
-                for (int rb = 0; rb < RB; ++rb) {
-                    const int n = rb * 128 + r;
-                    if (n >= N) continue;
-                    float mm = -INFINITY, ll = 0.0f;
-                    for (int g2 = 0; g2 < 4; ++g2) {  // fixed merge order
-                        const float2 p = sm.red[g2][n];
-                        const float mx = fmaxf(mm, p.x);
-                        const float x = (mm == -INFINITY) ? 0.0f : ll * ex2(mm - mx);
-                        const float y = (p.x == -INFINITY) ? 0.0f : p.y * ex2(p.x - mx);
-                        mm = mx;
-                        ll = x + y;
-                    }
-                    part[((size_t)bg * nsplit + split) * N + n] = make_float2(mm, ll);
-                }
-        } else {
-            // Thread owns token r of the tile and the heads g = cg, cg + 4, ...; head g's
-            // query rows are the columns [g*qe, (g+1)*qe), summed in row order.
-            for (int it = 0; it < count; ++it) {
-                const int a = it & 1;
-                ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                tc_fence_after();
-                const int t = tile_at(it) * kTile + r;
-                for (int g = cg; g < G; g += 4) {
-                    const int c0 = g * qe, c1 = c0 + qe;
-                    float acc = 0.0f;
-                    for (int cs = c0 & ~15; cs < c1; cs += 16) {
-                        uint32_t v[16];
-                        tmem_ld16(tmem + a * acc_cols + cs + lo, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int n = cs + e;
-                            if (n < c0 || n >= c1) continue;
-                            const float2 st = sm.stat[n];
-                            if (t <= pmin + (n - c0))
-                                acc = fmaf(ex2(fmaf(__uint_as_float(v[e]), sl2, -st.x)), st.y, acc);
-                        }
-                    }
-                    if (t < L) s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
-                }
-                tc_fence_before();
-                mbar_arrive(&sm.acc_empty[a]);
+        }
+        named_barrier(1, kEpiWarps * 32);
+        ok = __all_sync(0xffffffffu, ok) && !*abort;
+        if (ok && cg == 0)
+            for (int rb = 0; rb < RB; ++rb) {
+                const int n = rb * 128 + r;
+                if (n >= N) continue;
+                float mm = -INFINITY, ll = 0.0f;
+                for (int g2 = 0; g2 < 4; ++g2)  // fixed merge order
+                    online_merge(mm, ll, sm.red[g2][n].x, sm.red[g2][n].y);
+                __stcg(&part[((size_t)bg * nsplit + split) * N + n], make_float2(mm, ll));
             }
+        // ---- grid barrier: every CTA's pass-1 pairs are in global memory
+        __threadfence();
+        named_barrier(1, kEpiWarps * 32);
+        if (et == 0) {
+            int good = 0;
+            if (!*abort) {
+                atomicAdd(gbar, 1u);
+                const uint64_t t0 = globaltimer_ns();
+                for (uint32_t k = 0;; ++k) {
+                    unsigned v;
+                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gbar) : "memory");
+                    if (v >= nctas) { good = 1; break; }
+                    if ((k & 63) == 63 && (*abort || globaltimer_ns() - t0 > limit_ns)) break;
+                    __nanosleep(64);
+                }
+            }
+            sm.gbar_ok = good;
+        }
+        named_barrier(1, kEpiWarps * 32);
+        ok = ok && sm.gbar_ok;
+        // ---- merge the pass-1 pairs of this group in split order: (max, 1/sum) per row
+        if (ok && et < N) {
+            float mm = -INFINITY, ll = 0.0f;
+            for (int s = 0; s < nsplit; ++s) {
+                const float2 p = __ldcg(&part[((size_t)bg * nsplit + s) * N + et]);
+                online_merge(mm, ll, p.x, p.y);
+            }
+            sm.stat[et] = make_float2(mm, 1.0f / ll);
+        }
+        named_barrier(1, kEpiWarps * 32);
+        // ---- pass 2: thread owns token r of the tile and the heads g = cg, cg + 4, ...;
+        // head g's query rows are the columns [g*qe, (g+1)*qe), summed in row order.
+        for (int it = count; it < total && ok; ++it) {
+            const int a = it & 1;
+            ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            const int t = tile_at(it) * kTile + r;
+            for (int g = cg; g < G; g += 4) {
+                const int c0 = g * qe, c1 = c0 + qe;
+                float acc = 0.0f;
+                for (int cs = c0 & ~15; cs < c1; cs += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + a * 256 + cs + lo, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int n = cs + e;
+                        if (n < c0 || n >= c1) continue;
+                        const float2 st = sm.stat[n];
+                        if (t <= pmin + (n - c0))
+                            acc = fmaf(ex2(fmaf(__uint_as_float(v[e]), sl2, -st.x)), st.y, acc);
+                    }
+                }
+                if (t < L) s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty[a]);
         }
     }
     if (!ok) {
         *abort = 1;
-        report_error(ctl, TSA_ERR_DEVICE_TIMEOUT, (kPass2 ? 300 : 200) + warp);
+        report_error(ctl, TSA_ERR_DEVICE_TIMEOUT, 200 + warp);
     }
     tc_fence_before();
     __syncthreads();
@@ -316,14 +352,13 @@ int sm_count() {
 
 }  // namespace
 
-// Splits per KV group of the tensor-core scoring: about one CTA per SM in total.
+// Splits per KV group of the tensor-core scoring: about one CTA per SM in total (one
+// cooperative launch covers at most sm_count() groups).
 int score_tc_splits(const tsa_dims &dm) {
     const int ntiles = ceil_div(dm.L, kTile);
-    return std::max(1, std::min(ntiles, std::min(256, sm_count() / std::max(1, dm.B * dm.Hkv))));
+    const int groups = std::min(dm.B * dm.Hkv, sm_count());
+    return std::max(1, std::min(ntiles, std::min(256, sm_count() / groups)));
 }
-
-cudaError_t launch_combine(const float2 *part, int nsplit, int N, float2 *stat, int groups,
-                           cudaStream_t st);
 
 template <int D>
 static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *K, int qe,
@@ -338,29 +373,30 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
     // At least 116 KB so that one CTA holds an SM (and all 512 TMEM columns) at a time.
     const size_t smem = std::max<size_t>(sizeof(ScoreSmem<D>) + 1024, 116 * 1024);
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k_score_tc<D, false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+    if ((e = cudaFuncSetAttribute(k_score_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)))
         return e;
-    if ((e = cudaFuncSetAttribute(k_score_tc<D, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-        return e;
-    const int nsplit = score_tc_splits(dm);
-    const float sl2 = scale * 1.4426950408889634f;
+    int nsplit = score_tc_splits(dm);
+    float sl2 = scale * 1.4426950408889634f;
     float2 *part = reinterpret_cast<float2 *>(ws + w.score_part);
-    float2 *stat = reinterpret_cast<float2 *>(ws + w.score_stat);
     Control *ctl = reinterpret_cast<Control *>(ws);
-    const uint64_t lim = (uint64_t)limit_us * 1000ull;
-    dim3 grid(nsplit, dm.B * dm.Hkv);
-    k_score_tc<D, false><<<grid, kThreads, smem, st>>>(tk, (const __nv_bfloat16 *)Q, dm.L, dm.H,
-                                                       dm.Hkv, qe, sl2, nsplit, part, stat,
-                                                       s_h, ctl, lim, test_stall());
-    if ((e = cudaGetLastError())) return e;
-    const int N = (dm.H / dm.Hkv) * qe;
-    if ((e = launch_combine(part, nsplit, N, stat, dm.B * dm.Hkv, st))) return e;
-    k_score_tc<D, true><<<grid, kThreads, smem, st>>>(tk, (const __nv_bfloat16 *)Q, dm.L, dm.H,
-                                                      dm.Hkv, qe, sl2, nsplit, part, stat,
-                                                      s_h, ctl, lim, test_stall());
-    return cudaGetLastError();
+    unsigned int *gbar = reinterpret_cast<unsigned int *>(&ctl->pad[0]);
+    uint64_t lim = (uint64_t)limit_us * 1000ull;
+    int stall = test_stall();
+    const __nv_bfloat16 *Qb = (const __nv_bfloat16 *)Q;
+    int L = dm.L, H = dm.H, Hkv = dm.Hkv;
+    const int groups = dm.B * dm.Hkv, per_launch = std::min(groups, sm_count());
+    for (int g0 = 0; g0 < groups; g0 += per_launch) {
+        int group0 = g0;
+        const int gc = std::min(per_launch, groups - g0);
+        if ((e = cudaMemsetAsync(gbar, 0, sizeof(unsigned int), st))) return e;
+        void *args[] = {&tk, (void *)&Qb, &L, &H, &Hkv, &qe, &sl2, &nsplit, &group0,
+                        (void *)&part, (void *)&s_h, (void *)&gbar, (void *)&ctl, &lim, &stall};
+        e = cudaLaunchCooperativeKernel((const void *)k_score_tc<D>, dim3(nsplit, gc),
+                                        dim3(kThreads), args, smem, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_score_tc(const tsa_dims &dm, const void *Q, const void *K, int qe,
