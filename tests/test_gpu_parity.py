@@ -323,3 +323,17 @@ def test_attention_is_deterministic():
         assert torch.equal(tsa.tsa_attn(dm, Qh, Kh, Vh, Lk, ws=ws)[:, :, :lk], ref)
         assert torch.equal(tsa.tsa_attn(dm, x["Q"], x["K"], x["V"], None, dense=True, ws=ws), refd)
     assert tsa.tsa_get_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("H,Hkv,q,L", [(8, 1, 16, 2000),    # 128 query columns per group
+                                       (16, 1, 16, 1500),   # 256: query rows on the lanes
+                                       (8, 2, 64, 1300),    # q = 64 (the sweep's larger q)
+                                       (6, 2, 7, 777),      # odd sizes: 21 columns
+                                       (4, 4, 16, 3000)])   # MHA (one head per group)
+def test_scoring_shapes(H, Hkv, q, L):
+    x = make_inputs(1, L, H, Hkv, 128, torch.bfloat16, seed=H * 100 + q)
+    d = _dev(x)
+    s_h, s_l = tsa.tsa_score(d["Q"], d["K"], q)
+    ref_h, ref_l = oracle.score(x["Q"], x["K"], q)
+    assert_scores_close(s_h.cpu().numpy(), ref_h, "s_h")
+    assert_scores_close(s_l.cpu().numpy(), ref_l, "s_l")
