@@ -57,6 +57,17 @@ def _traffic(kernel: str, workload: str):
     return e["bytes_per_launch"] if h == e["source_sha"] else None
 
 
+def kv_union_rows(idx, lk: int, Hkv: int) -> int:
+    """Rows of K (and of V) a gather must read: per KV head, the tokens kept by at least
+    one of its query heads (idx is [B, H, L], its first lk entries per row kept)."""
+    import torch
+    B, H, L = idx.shape
+    kept = idx[:, :, :lk].reshape(B, Hkv, (H // Hkv) * lk).long()
+    mask = torch.zeros(B, Hkv, L, dtype=torch.bool, device=idx.device)
+    mask.scatter_(2, kept, True)
+    return int(mask.sum().item())
+
+
 def rank_seed(seed: int, rank: int) -> int:
     """Each rank draws its own sequence (batch sharding)."""
     return seed * 1000 + rank
@@ -220,6 +231,7 @@ def run_ours(args, w, L, rank, world, local_rank):
     ws = tsa.workspace(dm, w.q, layer=True, device=dev)
     Y = torch.empty_like(d["X"])
     Lk = torch.empty(1, dtype=torch.int32, device=dev)
+    idx = torch.empty(1, w.H, L, dtype=torch.int32, device=dev)
     st = torch.cuda.current_stream(dev)
 
     def sync_all():
@@ -234,7 +246,8 @@ def run_ours(args, w, L, rank, world, local_rank):
         for e in row:
             e.record(st)  # materialise the event handles
     for _ in range(args.warmup):
-        tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk, ws=ws)
+        tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk, idx=idx,
+                      ws=ws)
     sync_all()
     if tsa.tsa_get_device_status(ws) != 0:
         raise RuntimeError("device error during warm-up")
@@ -245,8 +258,8 @@ def run_ours(args, w, L, rank, world, local_rank):
         sync_all()
         t_start.record(st)
         for s in range(args.steps):
-            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk, ws=ws,
-                          stage_events=evs[s])
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk,
+                          idx=idx, ws=ws, stage_events=evs[s])
         t_stop.record(st)
         sync_all()
     total_ms = t_start.elapsed_time(t_stop)
@@ -272,7 +285,10 @@ def run_ours(args, w, L, rank, world, local_rank):
     H, dd = w.H, w.d
     hbm = {
         "score": (L * w.Hkv * dd * 2 + w.q * H * dd * 2 + 4 * H * L + 4 * L),
-        "gather": 6 * H * lk * dd * 2,
+        # Q rows read and Qh, Kh, Vh written once per query head; K and V rows read once
+        # per KV head over the union of its query heads' kept sets (the shared rows are
+        # L2 hits)
+        "gather": 4 * H * lk * dd * 2 + 2 * kv_union_rows(idx, lk, w.Hkv) * dd * 2,
         "scatter": 2 * L * H * dd * 2 + H * lk * dd * 2 + 4 * H * L,
     }
     hbm_roof = {k: {"ms": stage_ms[k], "achieved_gbs": v / (stage_ms[k] * 1e-3) / 1e9,

@@ -114,10 +114,12 @@ TSA_API tsa_status tsa_select(const tsa_dims *dims, const float *s_h, const int3
  * For i < Lkeep[b]: Qh[b,h,i] = Q[b,idx[b,h,i],h], Kh[b,h,i] = K[b,idx[b,h,i],kv(h)],
  * Vh likewise.  Rows i in [Lkeep[b], min(L, ceil128(Lkeep[b]))) of Qh, Kh, Vh are
  * zero-filled (the attention kernel reads whole 128-row tiles); later rows are not
- * written. */
+ * written.  An index outside [0, L) is skipped and reported as TSA_ERR_INVALID_ARG in the
+ * workspace's error word (ws supplies only the error word). */
 TSA_API tsa_status tsa_gather_qkv(const tsa_dims *dims, const void *Q, const void *K,
                           const void *V, const int32_t *idx, const int32_t *Lkeep,
-                          void *Qh, void *Kh, void *Vh, void *stream);
+                          void *Qh, void *Kh, void *Vh, void *ws, size_t ws_bytes,
+                          void *stream);
 
 /* Attention ([notes] 整体框架; [blog] §1.1 softmax(Q̂K̂ᵀ/√d)V̂).
  * dense == 0 (compressed): for each (b, h) and i < Lkeep[b],
@@ -171,7 +173,7 @@ TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K,
  * until the process exits.  The caller still passes Q, K, s_h and s_l.
  *   Limit   dims and q whose scoring workspace (tsa_workspace_size) exceeds 2 MiB are
  *           rejected with TSA_ERR_WORKSPACE before any device work; for example
- *           B = 1, L = 131072, 32/8 heads, q = 16 needs about 240 KB.
+ *           B = 1, L = 131072, 32/8 heads, q = 16 needs about 540 KB.
  *   Set-up  the first call on each device looks up the array's device address (with
  *           that device current) and caches it; make that first call before any stream
  *           capture.

@@ -98,8 +98,9 @@ def test_gather_attn_scatter_layer_validation():
     dm = _d()
     L = tsa.lib()
     f = [P(FAKE)] * 8
-    assert L.tsa_gather_qkv(ctypes.byref(dm), P(0), *f[:7], None) == 1
-    assert L.tsa_gather_qkv(ctypes.byref(dm), *f[:7], P(FAKE + 2), None) == 2
+    assert L.tsa_gather_qkv(ctypes.byref(dm), P(0), *f[:7], P(FAKE * 16), 4096, None) == 1
+    assert L.tsa_gather_qkv(ctypes.byref(dm), *f[:7], P(FAKE + 2), P(FAKE * 16), 4096, None) == 2
+    assert L.tsa_gather_qkv(ctypes.byref(dm), *f[:8], P(FAKE * 16), 8, None) == 4
     assert L.tsa_attn(ctypes.byref(dm), P(FAKE), P(FAKE), P(FAKE), P(0), 0, 0.088, P(FAKE),
                       P(FAKE * 16), 4096, None) == 1      # compressed mode needs Lkeep
     assert L.tsa_attn(ctypes.byref(dm), P(FAKE), P(FAKE), P(FAKE), None, 1, -1.0, P(FAKE),

@@ -39,7 +39,7 @@ def _stage_inputs():
     s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
     Lk = tsa.tsa_budget(dm, s_l, 0.02, ws=ws)
     idx = tsa.tsa_select(dm, s_h, Lk, ws=ws)
-    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk)
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk, ws=ws)
     assert tsa.tsa_get_device_status(ws) == 0
     return d, dm, Lk, Qh, Kh, Vh, s_h, s_l
 

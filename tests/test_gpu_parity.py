@@ -46,7 +46,7 @@ def run_stages(x, q, tau, in_place=False, Lkeep_override=None):
     if Lkeep_override is not None:
         Lk = torch.tensor(Lkeep_override, dtype=torch.int32, device="cuda")
     idx = tsa.tsa_select(dm, s_h, Lk, ws=ws)
-    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk)
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk, ws=ws)
     Oh = tsa.tsa_attn(dm, Qh, Kh, Vh, Lk, ws=ws)
     if in_place:
         Y = d["X"].clone()
@@ -315,7 +315,7 @@ def test_attention_is_deterministic():
     s_h, s_l = tsa.tsa_score(x["Q"], x["K"], 16, ws=ws)
     Lk = tsa.tsa_budget(dm, s_l, 0.005, ws=ws)
     idx = tsa.tsa_select(dm, s_h, Lk, ws=ws)
-    Qh, Kh, Vh = tsa.tsa_gather_qkv(x["Q"], x["K"], x["V"], idx, Lk)
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(x["Q"], x["K"], x["V"], idx, Lk, ws=ws)
     lk = int(Lk.item())
     ref = tsa.tsa_attn(dm, Qh, Kh, Vh, Lk, ws=ws)[:, :, :lk].clone()
     refd = tsa.tsa_attn(dm, x["Q"], x["K"], x["V"], None, dense=True, ws=ws).clone()

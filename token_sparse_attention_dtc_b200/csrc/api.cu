@@ -20,10 +20,11 @@ cudaError_t launch_norm(const tsa_dims &, const float *, float *, const WsLayout
                         cudaStream_t);
 cudaError_t launch_budget(const tsa_dims &, const float *, double, int32_t *, char *,
                           cudaStream_t);
-cudaError_t launch_select(const tsa_dims &, const float *, const int32_t *, int32_t *,
-                          Control *, cudaStream_t);
+cudaError_t launch_select(const tsa_dims &, const float *, const int32_t *, int32_t *, char *,
+                          cudaStream_t);
 cudaError_t launch_gather(const tsa_dims &, const void *, const void *, const void *,
-                          const int32_t *, const int32_t *, void *, void *, void *, cudaStream_t);
+                          const int32_t *, const int32_t *, void *, void *, void *, Control *,
+                          cudaStream_t);
 cudaError_t launch_attn_simt(const tsa_dims &, const void *, const void *, const void *,
                              const int32_t *, int, float, void *, cudaStream_t);
 cudaError_t launch_attn_tc(const tsa_dims &, const void *, const void *, const void *,
@@ -106,18 +107,17 @@ WsLayout ws_layout(const tsa_dims &dm, int q) {
     WsLayout w;
     w.qe = q < dm.L ? q : dm.L;
     w.N = (dm.H / dm.Hkv) * w.qe;
-    // splits per KV group: the CUDA-core path uses ceil(L / 4096), the tensor-core path
-    // at most min(#128-token tiles, 256)
-    w.nsplit = std::max(ceil_div(dm.L, kScoreSplitTokens), std::min(ceil_div(dm.L, 128), 256));
+    w.nsplit = score_split_cap(dm);
     w.nblk_norm = ceil_div(dm.L, 256);
-    size_t off = budget_end(dm.B);  // control block, budget state and histograms first
+    size_t off = align256(sizeof(Control));  // scoring scratch after the control block
     w.score_part = off;
     off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.nsplit * w.N);
     w.score_stat = off;
     off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.N);
     w.norm_part = off;
     off = align256(off + sizeof(float) * (size_t)dm.B * w.nblk_norm);
-    w.total = off;
+    // the budget and selection scratch overlap the scoring scratch (stages run in order)
+    w.total = std::max(off, std::max(budget_end(dm.B), select_end(dm.B, dm.H, dm.L)));
     return w;
 }
 
@@ -223,14 +223,14 @@ tsa_status tsa_select(const tsa_dims *dims, const float *s_h, const int32_t *Lke
     TSA_TRY(check_ptr(s_h, "s_h"));
     TSA_TRY(check_ptr(Lkeep, "Lkeep"));
     TSA_TRY(check_ptr(idx, "idx"));
-    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
-    return cuda_status(
-        launch_select(*dims, s_h, Lkeep, idx, (Control *)ws, (cudaStream_t)stream), "tsa_select");
+    TSA_TRY(check_ws(ws, ws_bytes, select_end(dims->B, dims->H, dims->L)));
+    return cuda_status(launch_select(*dims, s_h, Lkeep, idx, (char *)ws, (cudaStream_t)stream),
+                       "tsa_select");
 }
 
 tsa_status tsa_gather_qkv(const tsa_dims *dims, const void *Q, const void *K, const void *V,
                           const int32_t *idx, const int32_t *Lkeep, void *Qh, void *Kh, void *Vh,
-                          void *stream) {
+                          void *ws, size_t ws_bytes, void *stream) {
     TSA_TRY(check_dims(dims));
     TSA_TRY(check_ptr(Q, "Q"));
     TSA_TRY(check_ptr(K, "K"));
@@ -240,9 +240,10 @@ tsa_status tsa_gather_qkv(const tsa_dims *dims, const void *Q, const void *K, co
     TSA_TRY(check_ptr(Qh, "Qh"));
     TSA_TRY(check_ptr(Kh, "Kh"));
     TSA_TRY(check_ptr(Vh, "Vh"));
-    return cuda_status(
-        launch_gather(*dims, Q, K, V, idx, Lkeep, Qh, Kh, Vh, (cudaStream_t)stream),
-        "tsa_gather_qkv");
+    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
+    return cuda_status(launch_gather(*dims, Q, K, V, idx, Lkeep, Qh, Kh, Vh, (Control *)ws,
+                                     (cudaStream_t)stream),
+                       "tsa_gather_qkv");
 }
 
 tsa_status tsa_attn(const tsa_dims *dims, const void *Qh, const void *Kh, const void *Vh,
@@ -317,9 +318,10 @@ tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const v
     TSA_TRY(rec(1));
     TSA_TRY(cuda_status(launch_budget(dm, s_l, tau, Lk, w, st), "tsa_layer budget"));
     TSA_TRY(rec(2));
-    TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, (Control *)w, st), "tsa_layer select"));
+    TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, w, st), "tsa_layer select"));
     TSA_TRY(rec(3));
-    TSA_TRY(cuda_status(launch_gather(dm, Q, K, V, idx, Lk, Qh, Kh, Vh, st), "tsa_layer gather"));
+    TSA_TRY(cuda_status(launch_gather(dm, Q, K, V, idx, Lk, Qh, Kh, Vh, (Control *)w, st),
+                        "tsa_layer gather"));
     TSA_TRY(rec(4));
     TSA_TRY(do_attn(dm, Qh, Kh, Vh, Lk, 0, scale, Oh, w, st));
     TSA_TRY(rec(5));

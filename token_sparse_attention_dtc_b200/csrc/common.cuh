@@ -75,7 +75,20 @@ __host__ __device__ inline size_t budget_end(int B) {
     return align256(budget_hist_offset(B) + kBudgetHistBytes * (size_t)B);
 }
 
-// Layout of the workspace regions used by the stage kernels.
+// Top-k search state of one (batch, head) row of the selection.
+struct SelectState {
+    uint32_t prefix;   // key digits chosen so far; the threshold key at the end
+    int32_t need;      // tokens still to take from the current digit range
+    int32_t identity;  // 1 when L' is 0 or L (the index list is the identity)
+    int32_t pad;
+};
+static_assert(sizeof(SelectState) == 16, "select state is 16 bytes");
+size_t select_end(int B, int H, int L);
+
+// Every stage's scratch starts right after the 256-byte control block: the stages of a
+// layer run one after another on one stream and keep their results outside the scratch,
+// so their scratch regions may overlap.
+// Layout of the workspace regions used by the scoring kernels.
 struct WsLayout {
     size_t control = 0;     // Control
     size_t score_part = 0;  // float2 [B*Hkv][nsplit][N]  per-split (max, sum) in log2 units
@@ -86,6 +99,17 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const tsa_dims &dm, int q);
+
+// Capacity, per KV group, of the workspace's scoring splits: the CUDA-core path uses
+// ceil(L / 4096) splits, the tensor-core path at most ceil(256 / (B*Hkv)) (and no more
+// than the number of 128-token tiles).
+inline int score_split_cap(const tsa_dims &dm) {
+    const int groups = dm.B * dm.Hkv;
+    const int tc = ceil_div(256, groups) < ceil_div(dm.L, 128) ? ceil_div(256, groups)
+                                                              : ceil_div(dm.L, 128);
+    const int simt = ceil_div(dm.L, kScoreSplitTokens);
+    return simt > tc ? simt : tc;
+}
 
 // Host: the failure-path test hook set by tsa_set_test_stall (0 or 1).
 int test_stall();

@@ -20,7 +20,8 @@ template <int VPR>
 __global__ void __launch_bounds__(kMoveThreads)
 k_gather_qkv(const uint4 *__restrict__ Q, const uint4 *__restrict__ K, const uint4 *__restrict__ V,
              const int32_t *__restrict__ idx, const int32_t *__restrict__ Lkeep, int L, int H,
-             int Hkv, uint4 *__restrict__ Qh, uint4 *__restrict__ Kh, uint4 *__restrict__ Vh) {
+             int Hkv, uint4 *__restrict__ Qh, uint4 *__restrict__ Kh, uint4 *__restrict__ Vh,
+             Control *ctl) {
     const int bh = blockIdx.x, b = bh / H, h = bh % H, kv = h / (H / Hkv);
     const int Lk = Lkeep[b];
     const int pad_end = min(L, (Lk + 127) & ~127);
@@ -33,6 +34,10 @@ k_gather_qkv(const uint4 *__restrict__ Q, const uint4 *__restrict__ K, const uin
         const size_t dst = ((size_t)bh * L + i) * VPR + v;
         if (i < Lk) {
             const int t = S[i];
+            if ((unsigned)t >= (unsigned)L) {  // not an index list of this sequence
+                report_error(ctl, TSA_ERR_INVALID_ARG, 20);
+                continue;
+            }
             const size_t qs = (((size_t)b * L + t) * H + h) * VPR + v;
             const size_t ks = (((size_t)b * L + t) * Hkv + kv) * VPR + v;
             const uint4 q = Q[qs], k = K[ks], w = V[ks];
@@ -126,14 +131,14 @@ k_residual_dense(const uint4 *__restrict__ O, const uint4 *X, uint4 *Y, size_t n
 
 cudaError_t launch_gather(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                           const int32_t *idx, const int32_t *Lkeep, void *Qh, void *Kh, void *Vh,
-                          cudaStream_t st) {
+                          Control *ctl, cudaStream_t st) {
     const int esz = dm.dtype == TSA_F32 ? 4 : 2;
     const int vpr = dm.d * esz / 16;
     dim3 grid(dm.B * dm.H, ceil_div(dm.L, kGatherRows));
 #define TSA_GATHER(V_)                                                                        \
     k_gather_qkv<V_><<<grid, kMoveThreads, 0, st>>>(                                         \
         (const uint4 *)Q, (const uint4 *)K, (const uint4 *)V, idx, Lkeep, dm.L, dm.H, dm.Hkv, \
-        (uint4 *)Qh, (uint4 *)Kh, (uint4 *)Vh)
+        (uint4 *)Qh, (uint4 *)Kh, (uint4 *)Vh, ctl)
     switch (vpr) {
         case 8: TSA_GATHER(8); break;
         case 16: TSA_GATHER(16); break;

@@ -357,7 +357,8 @@ int sm_count() {
 int score_tc_splits(const tsa_dims &dm) {
     const int ntiles = ceil_div(dm.L, kTile);
     const int groups = std::min(dm.B * dm.Hkv, sm_count());
-    return std::max(1, std::min(ntiles, std::min(256, sm_count() / groups)));
+    const int n = std::max(1, std::min(ntiles, sm_count() / groups));
+    return std::min(n, score_split_cap(dm));  // never more than the workspace holds
 }
 
 template <int D>

@@ -53,7 +53,7 @@ def lib():
             "tsa_score": (I32, [DP, P, P, I32, F, P, P, P, SZ, P]),
             "tsa_budget": (I32, [DP, P, D, P, P, SZ, P]),
             "tsa_select": (I32, [DP, P, P, P, P, SZ, P]),
-            "tsa_gather_qkv": (I32, [DP, P, P, P, P, P, P, P, P, P]),
+            "tsa_gather_qkv": (I32, [DP, P, P, P, P, P, P, P, P, P, SZ, P]),
             "tsa_attn": (I32, [DP, P, P, P, P, I32, F, P, P, SZ, P]),
             "tsa_scatter_residual": (I32, [DP, P, P, P, P, P, P]),
             "tsa_layer": (I32, [DP, P, P, P, P, P, I32, I32, D, F, P, P, P, P, P, SZ, P, P]),
@@ -174,15 +174,17 @@ def tsa_select(dm: Dims, s_h, Lkeep, idx=None, ws=None, stream=None):
     return idx
 
 
-def tsa_gather_qkv(Q, K, V, idx, Lkeep, Qh=None, Kh=None, Vh=None, stream=None):
+def tsa_gather_qkv(Q, K, V, idx, Lkeep, Qh=None, Kh=None, Vh=None, ws=None, stream=None):
     dm = dims(Q, K)
     _need_cuda(Q, K, V, idx, Lkeep)
     shape = (dm.B, dm.H, dm.L, dm.d)
     Qh = torch.empty(shape, dtype=Q.dtype, device=Q.device) if Qh is None else Qh
     Kh = torch.empty(shape, dtype=Q.dtype, device=Q.device) if Kh is None else Kh
     Vh = torch.empty(shape, dtype=Q.dtype, device=Q.device) if Vh is None else Vh
+    if ws is None:
+        ws = workspace(dm, 1, device=Q.device)
     _check(lib().tsa_gather_qkv(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(idx), _p(Lkeep),
-                                _p(Qh), _p(Kh), _p(Vh), _stream(stream)))
+                                _p(Qh), _p(Kh), _p(Vh), _p(ws), ws.numel(), _stream(stream)))
     return Qh, Kh, Vh
 
 
