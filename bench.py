@@ -57,6 +57,16 @@ def _traffic(kernel: str, workload: str):
     return e["bytes_per_launch"] if h == e["source_sha"] else None
 
 
+def l2_note(d) -> str:
+    """Whether the timed inputs exceed the 126 MB L2 (no flush is done between steps)."""
+    mb = {k: d[k].numel() * d[k].element_size() / 1e6 for k in ("Q", "K", "V", "X")}
+    big = all(v > 126 for v in mb.values())
+    return ("inputs larger than L2 (Q %.0f MB, K/V %.0f MB each, X %.0f MB); no flush"
+            % (mb["Q"], mb["K"], mb["X"]) if big else
+            "inputs not all larger than L2 (Q %.0f MB, K/V %.0f MB each, X %.0f MB); no flush"
+            % (mb["Q"], mb["K"], mb["X"]))
+
+
 def kv_union_rows(idx, lk: int, Hkv: int) -> int:
     """Rows of K (and of V) a gather must read: per KV head, the tokens kept by at least
     one of its query heads (idx is [B, H, L], its first lk entries per row kept)."""
@@ -256,11 +266,13 @@ def run_ours(args, w, L, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         time.sleep(0.3)
         sync_all()
+        n_launch0 = tsa.kernel_launches()
         t_start.record(st)
         for s in range(args.steps):
             tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk,
                           idx=idx, ws=ws, stage_events=evs[s])
         t_stop.record(st)
+        n_launches = tsa.kernel_launches() - n_launch0
         sync_all()
     total_ms = t_start.elapsed_time(t_stop)
     ms_step = total_ms / args.steps
@@ -357,7 +369,6 @@ def run_ours(args, w, L, rank, world, local_rank):
         cpu = {"value": ms, "unit": "ms", "cores": info["threads"], "kind": "oracle",
                "sample": sample}
 
-    launches_per_step = 10  # score: 3 + 2 (normalise), budget, select, gather, attn, scatter
     if rank == 0:
         line = {
             "metric": METRIC, "value": ms_step / world, "unit": "ms", "n_gpus": world,
@@ -366,7 +377,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "data": "synthetic",
             "config": {"workload": _workload_desc(w, L), "global_batch": world, "seq_len": L,
                        "parallelism": "replicas (dp%d, no data-path collective)" % world,
-                       "l2": "inputs larger than L2 (Q 1.07 GB, K/V 268 MB each); no flush",
+                       "l2": l2_note(d),
                        "Lkeep": lk, "kept_fraction": lk / L},
             "roofline": roof,
             "stages_ms": stage_ms,
@@ -378,7 +389,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": n_launches,
             "peaks": peaks,
         }
         print(json.dumps(line), flush=True)

@@ -204,6 +204,11 @@ TSA_API void tsa_set_wait_limit(uint32_t microseconds);
  * down as described above, and exits.  Nothing faults, traps or hangs. */
 TSA_API void tsa_set_test_stall(int32_t on);
 
+/* Number of CUDA kernels this library has launched in this process, on every device and
+ * thread (a host-side counter; memset and copy operations are not counted).  Callers take
+ * the difference around a region to count its launches.  Never fails. */
+TSA_API uint64_t tsa_kernel_launches(void);
+
 TSA_API const char *tsa_status_string(tsa_status s);
 TSA_API const char *tsa_last_error(void);
 

@@ -113,6 +113,15 @@ def test_gather_attn_scatter_layer_validation():
                        None, P(FAKE * 16), 1 << 20, None, None) == 4
 
 
+def test_failed_validation_launches_nothing():
+    n0 = tsa.kernel_launches()
+    dm = _d()
+    assert _score(dm, Q=0) == 1
+    assert tsa.lib().tsa_select(ctypes.byref(dm), P(FAKE), P(FAKE), P(0), P(FAKE * 16), 4096,
+                                None) == 1
+    assert tsa.kernel_launches() == n0
+
+
 def test_status_strings():
     L = tsa.lib()
     for code, name in tsa.STATUS.items():

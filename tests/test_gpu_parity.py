@@ -230,6 +230,25 @@ def test_select_heavy_ties_bitexact():
         np.testing.assert_array_equal(idx.cpu().numpy(), oracle.select(s, lk))
 
 
+def test_select_multichunk_ties_bitexact():
+    """Several 4096-token chunks plus a ragged tail: tied runs at the threshold cross chunk
+    boundaries, keys span every digit range (zeros, denormals, values near the float
+    maximum), and one row is all-equal."""
+    rng = np.random.default_rng(7)
+    B, H, L = 2, 4, 3 * 4096 + 517
+    s = (rng.integers(0, 6, size=(B, H, L)) / 8).astype(np.float32)
+    s[0, 1] = np.float32(0.375)                                        # all equal
+    s[0, 2] = rng.choice(np.array([0.0, 1e-45, 1e-40, 1e-20, 1.0, 3e38], np.float32),
+                         size=L)
+    s[1, 3, 4000:4200] = np.float32(2.5)                               # run over a boundary
+    for keeps in ([1, L - 1], [L // 2, 4095], [4096, 4097], [4100, 8192], [L, 0],
+                  [rng.integers(1, L), rng.integers(1, L)]):
+        lk = np.array(keeps, np.int32)
+        dm = tsa.Dims(B, L, H, 1, 64, tsa.TSA_BF16)
+        idx = tsa.tsa_select(dm, torch.from_numpy(s).cuda(), torch.from_numpy(lk).cuda())
+        np.testing.assert_array_equal(idx.cpu().numpy(), oracle.select(s, lk), err_msg=str(keeps))
+
+
 def test_dense_attention_gqa_matches_oracle():
     x = make_inputs(2, 333, 8, 2, 128, torch.bfloat16, seed=9)
     d = _dev(x)

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <string>
 
 #include "common.cuh"
@@ -38,6 +39,9 @@ static uint32_t g_wait_limit_us = 2000000;  // 2 s
 static int g_test_stall = 0;
 
 int test_stall() { return g_test_stall; }
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 static tsa_status fail(tsa_status s, const char *fmt, ...) {
     char buf[512];
@@ -348,6 +352,8 @@ tsa_status tsa_get_device_status(void *ws, void *stream) {
 void tsa_set_wait_limit(uint32_t microseconds) { g_wait_limit_us = microseconds; }
 
 void tsa_set_test_stall(int32_t on) { g_test_stall = on ? 1 : 0; }
+
+uint64_t tsa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char *tsa_status_string(tsa_status s) {
     switch (s) {

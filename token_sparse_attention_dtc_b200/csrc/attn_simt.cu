@@ -129,6 +129,7 @@ static cudaError_t attn_simt_impl(const tsa_dims &dm, const void *Q, const void 
     k_attn_simt<T, D><<<(unsigned)nblocks, kAttnSimtThreads, smem, st>>>(
         (const T *)Q, (const T *)K, (const T *)V, Lkeep, dense, dm.L, dm.H, dm.Hkv,
         scale * 1.4426950408889634f, (T *)O);
+    note_launches(1);
     return cudaGetLastError();
 }
 

@@ -374,6 +374,7 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
     k_attn_tc<D><<<(unsigned)nblocks, kThreads, smem, st>>>(
         tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
         (__nv_bfloat16 *)O, ctl, (uint64_t)limit_us * 1000ull, test_stall());
+    note_launches(1);
     return cudaGetLastError();
 }
 

@@ -210,6 +210,7 @@ cudaError_t launch_budget(const tsa_dims &dm, const float *s_l, double tau, int3
     cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)dm.B * kBudgetHistBytes, stream);
     if (e != cudaSuccess) return e;
     k_budget_init<<<ceil_div(dm.B, 128), 128, 0, stream>>>(st, dm.B, T, Lkeep, dm.L);
+    note_launches(1 + 3 * 2);  // init, (histogram, scan) per level
     dim3 hg(ceil_div(dm.L, kHistThreads * kHistPerThread), dm.B);
     for (int lv = 0; lv < 3; ++lv) {
         const size_t smem = (size_t)12 << level_bits(lv);

@@ -85,6 +85,9 @@ struct SelectState {
 static_assert(sizeof(SelectState) == 16, "select state is 16 bytes");
 size_t select_end(int B, int H, int L);
 
+// Host-side count of kernels this library has launched (read by tsa_kernel_launches).
+void note_launches(int n);
+
 // Every stage's scratch starts right after the 256-byte control block: the stages of a
 // layer run one after another on one stream and keep their results outside the scratch,
 // so their scratch regions may overlap.

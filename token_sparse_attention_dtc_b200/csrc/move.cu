@@ -146,6 +146,7 @@ cudaError_t launch_gather(const tsa_dims &dm, const void *Q, const void *K, cons
         default: return cudaErrorInvalidValue;
     }
 #undef TSA_GATHER
+    note_launches(1);
     return cudaGetLastError();
 }
 
@@ -159,6 +160,7 @@ static cudaError_t scatter_impl(const tsa_dims &dm, const void *Oh, const int32_
                                                  (size_t)148 * 16);
         k_residual_dense<T><<<blocks, kMoveThreads, 0, st>>>((const uint4 *)Oh, (const uint4 *)X,
                                                             (uint4 *)Y, nvec);
+        note_launches(1);
         return cudaGetLastError();
     }
     dim3 grid(dm.B * dm.H, ceil_div(dm.L, kGatherRows));
@@ -177,6 +179,7 @@ static cudaError_t scatter_impl(const tsa_dims &dm, const void *Oh, const int32_
         default: return cudaErrorInvalidValue;
     }
 #undef TSA_SCATTER
+    note_launches(1);
     return cudaGetLastError();
 }
 

@@ -231,6 +231,7 @@ static cudaError_t score_simt_impl(const tsa_dims &dm, const void *Q, const void
     k_score_combine<<<dm.B * dm.Hkv, 256, 0, st>>>(part, nsplit, G * qe, stat);
     k_score_colsum_simt<T, D, kScoreSplitTokens / kSimtThreads><<<grid, kSimtThreads, 0, st>>>(
         (const T *)Q, (const T *)K, dm.L, dm.H, dm.Hkv, qe, sl2, split_len, stat, s_h);
+    note_launches(3);
     return cudaGetLastError();
 }
 
@@ -245,6 +246,7 @@ cudaError_t launch_score_simt(const tsa_dims &dm, const void *Q, const void *K, 
 cudaError_t launch_combine(const float2 *part, int nsplit, int N, float2 *stat, int groups,
                            cudaStream_t st) {
     k_score_combine<<<groups, 256, 0, st>>>(part, nsplit, N, stat);
+    note_launches(1);
     return cudaGetLastError();
 }
 
@@ -254,6 +256,7 @@ cudaError_t launch_norm(const tsa_dims &dm, const float *s_h, float *s_l, const 
     dim3 grid(w.nblk_norm, dm.B);
     k_norm_u<<<grid, 256, 0, st>>>(s_h, dm.L, dm.H, w.nblk_norm, s_l, part);
     k_norm_div<<<grid, 256, 0, st>>>(s_l, dm.L, w.nblk_norm, part);
+    note_launches(2);
     return cudaGetLastError();
 }
 

@@ -396,6 +396,7 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
         e = cudaLaunchCooperativeKernel((const void *)k_score_tc<D>, dim3(nsplit, gc),
                                         dim3(kThreads), args, smem, st);
         if (e != cudaSuccess) return e;
+        note_launches(1);
     }
     return cudaSuccess;
 }

@@ -285,6 +285,7 @@ cudaError_t launch_select(const tsa_dims &dm, const float *s_h, const int32_t *L
     unsigned int *hist = reinterpret_cast<unsigned int *>(ws + y.hist);
     ChunkInfo *ci = reinterpret_cast<ChunkInfo *>(ws + y.chunks);
     k_sel_init<<<ceil_div(rows, 256), 256, 0, stream>>>(Lkeep, dm.L, dm.H, rows, st, ctl);
+    note_launches(1 + 3 * 2 + 3);  // init, (histogram, scan) per level, count/offsets/write
     dim3 hg(ceil_div(dm.L, kHistThreads * kHistPerThread), rows);
     for (int lv = 0; lv < 3; ++lv) {
         cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)4096 * 4 * rows, stream);

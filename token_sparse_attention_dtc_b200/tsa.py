@@ -23,7 +23,8 @@ STATUS = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_ALIGNMENT",
 EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_budget",
            "tsa_select", "tsa_gather_qkv", "tsa_attn", "tsa_scatter_residual", "tsa_layer",
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
-           "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall")
+           "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall",
+           "tsa_kernel_launches")
 
 
 class TSAError(RuntimeError):
@@ -60,6 +61,7 @@ def lib():
             "tsa_get_device_status": (I32, [P, P]),
             "tsa_set_wait_limit": (None, [ctypes.c_uint32]),
             "tsa_set_test_stall": (None, [I32]),
+            "tsa_kernel_launches": (ctypes.c_uint64, []),
             "tsa_status_string": (ctypes.c_char_p, [I32]),
             "tsa_last_error": (ctypes.c_char_p, []),
             "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
@@ -238,6 +240,11 @@ def tsa_get_device_status(ws, stream=None) -> int:
 
 def tsa_set_wait_limit(microseconds: int):
     lib().tsa_set_wait_limit(int(microseconds))
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched so far in this process (host-side counter)."""
+    return int(lib().tsa_kernel_launches())
 
 
 def tsa_set_test_stall(on: bool):
