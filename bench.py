@@ -307,6 +307,13 @@ def run_ours(args, w, L, rank, world, local_rank):
                     "frac": v / (stage_ms[k] * 1e-3) / 1e9 / peaks["hbm"],
                     "algorithmic_bytes": v}
                 for k, v in hbm.items()}
+    # ncu-counted DRAM bytes of the committed capture, when it matches the source
+    for k, kern in (("score", "k_score_tc"), ("gather", "k_gather_qkv"),
+                    ("scatter", "k_scatter_residual")):
+        t = _traffic(kern, w.name)
+        hbm_roof[k]["traffic"] = t
+        hbm_roof[k]["dram_gbs"] = t / (stage_ms[k] * 1e-3) / 1e9 if t else None
+        hbm_roof[k]["dram_frac"] = (t / (stage_ms[k] * 1e-3) / 1e9 / peaks["hbm"]) if t else None
 
     # dense causal attention through the same kernel, same shape
     dense = None
