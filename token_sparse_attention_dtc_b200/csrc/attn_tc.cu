@@ -9,14 +9,14 @@
 //
 // One CTA per pair of 128-row query tiles (A = 2p, B = 2p+1) of one head; every K/V
 // tile is loaded once and used by both.  CTAs run head by head, heaviest pairs first.
-// Warp roles (384 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: both Q tiles once, then K and V tiles through a 2-stage ring.
 //   warp 1      TMEM owner and MMA issuer.  Order per key tile j:
 //                 PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
 //               so that the softmax of one tile overlaps the MMAs of the other.  S = Q K^T
 //               goes to the tile's TMEM S buffer; O += P V reads P (bf16, written over S)
 //               from TMEM and V from shared memory.
-//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: thread r owns query row r.
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B: thread r owns query row r.
 //               Online max/sum in log2 units; O is rescaled only when the running max grows
 //               by more than 2^8 (so P <= 2^8); P is written back to TMEM; the epilogue
 //               writes O / l as bf16.
@@ -36,7 +36,7 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kStages = 2, kThreads = 384;
+constexpr int kBM = 128, kBN = 128, kStages = 2, kThreads = 320;
 constexpr uint64_t kDrainNs = 1000000000ull;  // drain waits: 1 s
 
 template <int D> struct AttnSmem {
@@ -56,6 +56,34 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+
+// P = 2^(S*sl2 - mu) of one row, packed to bf16x2 over sr[0..63]; returns the row sum of
+// the fp32 values.  Paired fp32 instructions for the scale-subtract and the sums.
+// kDiag: the diagonal tile, whose masked entries are -inf and give exactly 0.  (The two
+// instantiations compile to the same arithmetic; keeping the diagonal step separate lets
+// the register allocator treat the common step on its own.)
+template <bool kDiag>
+__device__ __forceinline__ float exp_pack_row(uint32_t (&sr)[128], float sl2, float mu) {
+    const float nmu = -mu;
+    float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {  // columns 2c .. 2c+3 (pairs c and c+1)
+        float x0, x1, x2, x3, p0, p1, p2, p3;
+        fma2(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), sl2, sl2, nmu,
+             nmu);
+        fma2(x2, x3, __uint_as_float(sr[2 * c + 2]), __uint_as_float(sr[2 * c + 3]), sl2, sl2,
+             nmu, nmu);
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+        p2 = ex2(x2);
+        p3 = ex2(x3);
+        add2(a0, a1, a0, a1, p0, p1);
+        add2(b0, b1, b0, b1, p2, p3);
+        sr[c] = pack_bf16(p0, p1);  // in place: sr[c] and sr[c+1] were already read
+        sr[c + 1] = pack_bf16(p2, p3);
+    }
+    return (a0 + a1) + (b0 + b1);
 }
 
 // Softmax of one query tile (this warpgroup), steps j = 0..n-1; the last step is the
@@ -98,21 +126,8 @@ __device__ __forceinline__ bool softmax_tile(AttnSmem<D> &sm, int X, int n, uint
             resc = true;
         }
         m = mu;
-        float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), sl2, -mu));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), sl2, -mu));
-            const float p2 = ex2(fmaf(__uint_as_float(sr[2 * c + 2]), sl2, -mu));
-            const float p3 = ex2(fmaf(__uint_as_float(sr[2 * c + 3]), sl2, -mu));
-            s0 += p0;
-            s1 += p1;
-            s2 += p2;
-            s3 += p3;
-            sr[c] = pack_bf16(p0, p1);  // in place: sr[c] and sr[c+1] were already read
-            sr[c + 1] = pack_bf16(p2, p3);
-        }
-        l = l * factor + ((s0 + s1) + (s2 + s3));
+        l = l * factor +
+            (j == n - 1 ? exp_pack_row<true>(sr, sl2, mu) : exp_pack_row<false>(sr, sl2, mu));
         if (__any_sync(0xffffffffu, resc)) {
             // S_X(j) was issued after PV_X(j-1), so O_X is complete here.
             const float f = resc ? factor : 1.0f;
@@ -189,7 +204,6 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort = &sm.abort;
     bool ok = true;
-
     if (warp == 0) {
         if (lane == 0) {
             int issued = 0;  // K/V tiles issued (negative: K of tile -issued-1 only)
@@ -287,8 +301,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 mbar_wait(&sm.drain, 0, kDrainNs, &sm.never);
             }
         }
-    } else if (warp >= 4) {
-        const int X = (warp - 4) >> 2;  // 0: tile A (warps 4-7), 1: tile B (warps 8-11)
+    } else {
+        // 0: tile A (warps 2-5), 1: tile B (warps 6-9).  A warp reaches only the TMEM lane
+        // quadrant warp % 4, and any four consecutive warps cover all four.
+        const int X = (warp - 2) >> 2;
         const int wq = warp & 3, r = wq * 32 + lane;
         const uint32_t lo = (uint32_t)(wq * 32) << 16;
         const int n = X ? nB : nA;
