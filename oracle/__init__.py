@@ -47,8 +47,10 @@ def _load():
         lib.orc_select.argtypes = [I, I, I, P, P, P]
         lib.orc_attend_rows.argtypes = [I, I, I, I, I, I, P, P, P, P, P, D, L, P, P, I]
         lib.orc_decompress_residual.argtypes = [I, I, I, I, I, P, P, P, P, P, P]
+        lib.orc_budget_fixed.argtypes = [I, I, D, P]
+        lib.orc_pool.argtypes = [I, I, I, P, I, I, P, P]
         for f in ("orc_score", "orc_budget", "orc_select", "orc_attend_rows",
-                  "orc_decompress_residual"):
+                  "orc_decompress_residual", "orc_budget_fixed", "orc_pool"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -119,6 +121,32 @@ def budget(s_l, tau: float):
     if rc:
         raise ValueError("orc_budget rejected its arguments (%d)" % rc)
     return out, int(dis[0])
+
+
+def budget_fixed(B: int, L: int, sparsity: float):
+    """Fixed-ratio budget (ablation): L' = L - floor(sparsity * L) for every batch element."""
+    out = np.zeros(B, np.int32)
+    rc = _load().orc_budget_fixed(int(B), int(L), float(sparsity), _ptr(out))
+    if rc:
+        raise ValueError("orc_budget_fixed rejected its arguments (%d)" % rc)
+    return out
+
+
+POOL_MAX, POOL_MEAN = 1, 2
+
+
+def pool(s_h, kind: int, width: int):
+    """Token-axis pooling of head scores s_h [B, H, L] (any float dtype, taken exactly);
+    kind POOL_MAX or POOL_MEAN over the clipped window of odd `width`.  Returns
+    (pooled fp64 [B, H, L], s_l fp64 [B, L])."""
+    s = np.ascontiguousarray(_np(s_h), dtype=np.float64)
+    B, H, L = s.shape
+    out = np.zeros((B, H, L), np.float64)
+    sl = np.zeros((B, L), np.float64)
+    rc = _load().orc_pool(B, H, L, _ptr(s), int(kind), int(width), _ptr(out), _ptr(sl))
+    if rc:
+        raise ValueError("orc_pool rejected its arguments (%d)" % rc)
+    return out, sl
 
 
 def select(s_h, Lkeep):

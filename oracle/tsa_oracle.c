@@ -26,7 +26,8 @@
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   scoring is causal (recent query p sees keys t <= p) and uses the same
- *   1/sqrt(d) scale as attention; "pool" after the column sum adds nothing;
+ *   1/sqrt(d) scale as attention; "pool" after the column sum adds nothing in
+ *   the method as benchmarked (orc_pool gives the max / mean variants);
  *   "normalize" is division by the total; the coverage cumulative sum is taken
  *   in 2^-62 fixed point; top-k ties go to the lower token index; S_h is listed
  *   in ascending token order; GQA query head h reads KV head h / (H / Hkv).
@@ -215,6 +216,61 @@ int orc_budget(int B, int L, const float *s_l, double tau, int32_t *Lkeep,
     }
     free(v);
     if (real_disagree) *real_disagree = dis;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Budget variant for the ablation: a fixed sparsity ratio s instead of the  */
+/* coverage threshold.  [notes] 消融实验 (Fixed s = 0.3 / s = 0.5 against the  */
+/* dynamic budget) and 关键设计 2 (a one-size "cut 30%" is what the coverage  */
+/* budget replaces).  Reading: s is the fraction of tokens pruned, so        */
+/* k = floor(s * L) (in double) and L' = L - k, the same for every batch     */
+/* element.                                                                  */
+/* ------------------------------------------------------------------------ */
+int orc_budget_fixed(int B, int L, double s, int32_t *Lkeep) {
+    if (B < 1 || L < 1 || !(s >= 0.0 && s <= 1.0)) return 1;
+    const int k = (int)floor(s * (double)L);
+    for (int b = 0; b < B; ++b) Lkeep[b] = L - k;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Score variant: pooling of the head scores along the token axis.          */
+/* [notes] 关键设计 2: the column sums are pooled to give s_h before the     */
+/* layer score.  The pages name no pooling kind or window; the two plain     */
+/* readings are built: kind 1 = max, kind 2 = mean, over the window          */
+/* [t - r, t + r] (width = 2r + 1, odd) clipped to [0, L): the mean divides  */
+/* by the number of in-range tokens.  Then u[t] = sum_h pooled[t] and        */
+/* s_l = u / sum_t u, as in step 1.                                          */
+/* ------------------------------------------------------------------------ */
+int orc_pool(int B, int H, int L, const double *s_h, int kind, int width,
+             double *out, double *s_l) {
+    if (B < 1 || H < 1 || L < 1 || width < 1 || (width & 1) == 0 || (kind != 1 && kind != 2))
+        return 1;
+    const int rad = width / 2;
+    for (long row = 0; row < (long)B * H; ++row) {
+        const double *in = s_h + (size_t)row * L;
+        double *o = out + (size_t)row * L;
+        for (int t = 0; t < L; ++t) {
+            const int lo = t - rad < 0 ? 0 : t - rad, hi = t + rad > L - 1 ? L - 1 : t + rad;
+            double acc = kind == 1 ? -INFINITY : 0.0;
+            for (int u = lo; u <= hi; ++u) {
+                if (kind == 1) { if (in[u] > acc) acc = in[u]; }
+                else acc += in[u];
+            }
+            o[t] = kind == 1 ? acc : acc / (double)(hi - lo + 1);
+        }
+    }
+    for (int b = 0; b < B; ++b) {
+        double *sl = s_l + (size_t)b * L, tot = 0.0;
+        for (int t = 0; t < L; ++t) {
+            double u = 0.0;
+            for (int h = 0; h < H; ++h) u += out[((size_t)b * H + h) * L + t];
+            sl[t] = u;
+            tot += u;
+        }
+        for (int t = 0; t < L; ++t) sl[t] /= tot;
+    }
     return 0;
 }
 

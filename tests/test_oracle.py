@@ -304,3 +304,92 @@ def test_bf16_decode_matches_torch():
     O, Y = oracle.decompress_residual(np.zeros((1, 1, 1000, 1)), None, None,
                                       v.view(1, 1000, 1))
     np.testing.assert_array_equal(Y[0, :, 0], v.double().numpy())
+
+
+# ---------------------------------------------------------------- budget / score variants
+@pytest.mark.parametrize("L", [10, 1000, 131070])
+def test_budget_fixed_prunes_the_stated_decimal_fraction(L):
+    # The pages' ablation prunes a fixed 30% / 50%: s = m/10 removes exactly m*L/10 tokens.
+    for m in range(11):
+        lk = oracle.budget_fixed(2, L, m / 10)
+        assert list(lk) == [L - m * L // 10] * 2
+
+
+def test_budget_fixed_limits_and_rejects():
+    assert oracle.budget_fixed(1, 7, 0.0)[0] == 7
+    assert oracle.budget_fixed(1, 7, 1.0)[0] == 0
+    assert oracle.budget_fixed(1, 7, 0.5)[0] == 4          # floor(3.5) pruned
+    for bad in (-0.1, 1.5, float("nan")):
+        with pytest.raises(ValueError):
+            oracle.budget_fixed(1, 7, bad)
+
+
+def _pool_brute(s, kind, width):
+    """Pure-Python restatement on small inputs: clipped windows, index-order sums."""
+    r = width // 2
+    B, H, L = s.shape
+    out = np.zeros_like(s, dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for t in range(L):
+                w = [float(s[b, h, u]) for u in range(max(0, t - r), min(L, t + r + 1))]
+                out[b, h, t] = max(w) if kind == oracle.POOL_MAX else sum(w) / len(w)
+    return out
+
+
+@pytest.mark.parametrize("kind", [1, 2])
+def test_pool_width_one_is_identity(kind):
+    s = np.random.default_rng(0).random((2, 3, 17))
+    p, sl = oracle.pool(s, kind, 1)
+    np.testing.assert_array_equal(p, s)
+    np.testing.assert_allclose(sl, s.sum(1) / s.sum(1).sum(1, keepdims=True), rtol=1e-15)
+
+
+def test_pool_delta_gives_the_clipped_window():
+    L, w = 12, 5
+    for pos in (0, 1, 6, 11):
+        s = np.zeros((1, 1, L))
+        s[0, 0, pos] = 1.0
+        mx, _ = oracle.pool(s, oracle.POOL_MAX, w)
+        mean, _ = oracle.pool(s, oracle.POOL_MEAN, w)
+        for t in range(L):
+            inside = abs(t - pos) <= 2
+            cnt = min(L - 1, t + 2) - max(0, t - 2) + 1
+            assert mx[0, 0, t] == (1.0 if inside else 0.0)
+            assert mean[0, 0, t] == pytest.approx(1.0 / cnt if inside else 0.0, abs=0, rel=1e-15)
+
+
+def test_pool_mean_keeps_a_constant_at_the_edges():
+    s = np.full((1, 2, 9), 0.125)
+    p, sl = oracle.pool(s, oracle.POOL_MEAN, 7)
+    np.testing.assert_array_equal(p, s)          # 0.125 * n / n is exact
+    np.testing.assert_allclose(sl, 1.0 / 9, rtol=1e-15)
+
+
+@pytest.mark.parametrize("kind,width", [(1, 3), (1, 7), (2, 3), (2, 9)])
+def test_pool_matches_brute_force(kind, width):
+    s = np.random.default_rng(width + kind).random((2, 3, 23)).astype(np.float32)
+    p, sl = oracle.pool(s, kind, width)
+    np.testing.assert_allclose(p, _pool_brute(s, kind, width), rtol=1e-15, atol=0)
+    u = p.sum(1)
+    np.testing.assert_allclose(sl, u / u.sum(1, keepdims=True), rtol=1e-14)
+    np.testing.assert_allclose(sl.sum(1), 1.0, rtol=1e-14)
+
+
+def test_pool_mean_matches_prefix_sums_and_max_bounds():
+    s = np.random.default_rng(5).random((1, 1, 200))
+    r = 15
+    p, _ = oracle.pool(s, oracle.POOL_MEAN, 2 * r + 1)
+    c = np.concatenate([[0.0], np.cumsum(s[0, 0])])
+    lo = np.maximum(np.arange(200) - r, 0)
+    hi = np.minimum(np.arange(200) + r, 199)
+    np.testing.assert_allclose(p[0, 0], (c[hi + 1] - c[lo]) / (hi - lo + 1), rtol=1e-12)
+    mx, _ = oracle.pool(s, oracle.POOL_MAX, 2 * r + 1)
+    assert np.all(mx >= s) and np.all(mx >= p)
+
+
+def test_pool_rejects_bad_arguments():
+    s = np.ones((1, 1, 4))
+    for kind, width in ((3, 3), (1, 2), (2, 0)):
+        with pytest.raises(ValueError):
+            oracle.pool(s, kind, width)
