@@ -164,6 +164,55 @@ TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K,
                      int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
                      void *const *stage_events);
 
+/* ---- Budget and score variants ([notes] 消融实验 and 关键设计 2) ------------------- */
+
+typedef enum { TSA_POOL_NONE = 0, TSA_POOL_MAX = 1, TSA_POOL_MEAN = 2 } tsa_pool_kind;
+typedef enum { TSA_BUDGET_COVERAGE = 0, TSA_BUDGET_FIXED = 1 } tsa_budget_kind;
+
+/* Fixed-ratio budget, the ablation the notes compare the coverage budget with
+ * (消融实验, "Fixed s = 0.3 / 0.5"): `sparsity` is the fraction of tokens pruned, so
+ * Lkeep[b] = L - floor(sparsity * L) for every b (the product taken in double).
+ * sparsity in [0, 1], else TSA_ERR_INVALID_ARG.  Lkeep is [B] int32 on the device. */
+TSA_API tsa_status tsa_budget_fixed(const tsa_dims *dims, double sparsity, int32_t *Lkeep,
+                                    void *stream);
+
+/* Pooling of the head scores along the token axis ([notes] 关键设计 2: the column sums
+ * are pooled into s_h before the layer score; the pages name neither kind nor window):
+ *   s_h_out[b,h,t] = max or mean of s_h[b,h,u] over u in [t - r, t + r] clipped to
+ *   [0, L), width = 2r + 1; the mean divides by the number of tokens in range (fp32
+ *   sum in token order, one division).
+ * Then s_l_out[b,t] = u[t] / sum_t u with u[t] = sum_h s_h_out[b,h,t], as in tsa_score.
+ * kind TSA_POOL_MAX or TSA_POOL_MEAN; width odd, 1 <= width <= 255 (else
+ * TSA_ERR_INVALID_ARG / TSA_ERR_UNSUPPORTED).  s_h_out must not overlap s_h.  ws as for
+ * tsa_score with q = 1 (tsa_workspace_size(dims, 1) bytes). */
+TSA_API tsa_status tsa_pool_scores(const tsa_dims *dims, const float *s_h, int32_t kind,
+                                   int32_t width, float *s_h_out, float *s_l_out, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/* Options of tsa_layer_ex.  budget TSA_BUDGET_COVERAGE uses tau (as tsa_layer);
+ * TSA_BUDGET_FIXED uses sparsity (as tsa_budget_fixed).  pool TSA_POOL_NONE uses the
+ * scores as they are (as tsa_layer); otherwise selection and budget use the pooled head
+ * scores (as tsa_pool_scores with pool_width). */
+typedef struct {
+    int32_t budget;     /* tsa_budget_kind                      */
+    double tau;         /* coverage threshold, [0, 1)           */
+    double sparsity;    /* fixed fraction pruned, [0, 1]        */
+    int32_t pool;       /* tsa_pool_kind                        */
+    int32_t pool_width; /* odd, 1..255 (ignored for POOL_NONE)  */
+} tsa_layer_opts;
+
+/* tsa_layer with the budget and score variants of tsa_layer_opts (opts NULL: coverage
+ * budget with tau = 0.005, no pooling).  When pooling, s_h_out and s_l_out receive the
+ * pooled head scores and their layer score (the ones budget and selection used); the
+ * raw scores stay in ws.  Workspace: tsa_layer_workspace_size() bytes.  Everything else
+ * as tsa_layer. */
+TSA_API tsa_status tsa_layer_ex(const tsa_dims *dims, const void *Q, const void *K,
+                                const void *V, const void *X, void *Y, int32_t is_sparse,
+                                int32_t q, const tsa_layer_opts *opts, float scale,
+                                float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
+                                int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
+                                void *const *stage_events);
+
 /* Scoring for callers that cannot allocate device memory when they call in, such as an
  * engine whose device memory is fully planned up front by its own allocator, or a host
  * thread that must not enter the CUDA allocator.  Those callers cannot create the `ws`

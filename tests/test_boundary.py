@@ -113,6 +113,33 @@ def test_gather_attn_scatter_layer_validation():
                        None, P(FAKE * 16), 1 << 20, None, None) == 4
 
 
+def test_variant_validation():
+    dm = _d()
+    L = tsa.lib()
+    n0 = tsa.kernel_launches()
+    for s in (-0.1, 1.01, float("nan")):
+        assert L.tsa_budget_fixed(ctypes.byref(dm), s, P(FAKE), None) == 1
+    assert L.tsa_budget_fixed(ctypes.byref(dm), 0.3, P(0), None) == 1
+    assert L.tsa_budget_fixed(ctypes.byref(_d(L=0)), 0.3, P(FAKE), None) == 1
+    pool = lambda kind, width, out=FAKE * 64, wsb=1 << 30: L.tsa_pool_scores(
+        ctypes.byref(dm), P(FAKE), kind, width, P(out), P(FAKE), P(FAKE * 16), wsb, None)
+    assert pool(0, 3) == 1 and pool(3, 3) == 1 and pool(1, 4) == 1 and pool(2, -1) == 1
+    assert pool(1, 257) == 3
+    assert pool(1, 3, out=FAKE) == 1                    # output overlaps the input
+    assert pool(1, 3, wsb=8) == 4
+    opts = tsa.LayerOpts(7, 0.01, 0.0, 0, 1)              # unknown budget kind
+    ex = lambda o: L.tsa_layer_ex(ctypes.byref(dm), *[P(FAKE)] * 5, 1, 16, ctypes.byref(o),
+                                  0.088, None, None, None, None, P(FAKE * 16), 1 << 40, None,
+                                  None)
+    assert ex(opts) == 1
+    assert ex(tsa.LayerOpts(1, 0.01, 1.5, 0, 1)) == 1    # sparsity out of range
+    assert ex(tsa.LayerOpts(0, 0.01, 0.0, 2, 8)) == 1    # even pool width
+    assert ex(tsa.LayerOpts(0, 0.01, 0.0, 1, 301)) == 3  # pool width above 255
+    assert tsa.kernel_launches() == n0
+    # workspace: the layer holds the pooled scores too
+    assert tsa.workspace_size(dm, 16, layer=True) >= 2 * 4 * 32 * 4096 + 4 * 32 * 4096 * 128 * 2
+
+
 def test_failed_validation_launches_nothing():
     n0 = tsa.kernel_launches()
     dm = _d()

@@ -1,0 +1,121 @@
+"""GPU parity of the budget and score variants (fixed-ratio budget, pooled head scores)
+against the oracle, through the C ABI.
+
+Tolerances:
+  * fixed budget, max pooling, budget and selection on the GPU's scores: bit-exact;
+  * mean pooling: the fp32 sum of `width` positive terms in token order and one
+    division, against the fp64 mean of the same fp32 inputs: relative (width + 1) * 2^-23;
+  * layer scores s_l: relative 1e-5, as for the plain scores;
+  * attention and Y: as in test_gpu_parity.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from token_sparse_attention_dtc_b200 import tsa
+from token_sparse_attention_dtc_b200.inputs import make_inputs
+
+from test_gpu_parity import ATOL, HALF_ULP, assert_scores_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("L", [1, 1000, 131072])
+def test_budget_fixed_matches_oracle(L):
+    dm = tsa.Dims(3, L, 32, 8, 128, tsa.TSA_BF16)
+    for s in (0.0, 0.123, 0.3, 0.5, 0.999, 1.0):
+        lk = tsa.tsa_budget_fixed(dm, s)
+        np.testing.assert_array_equal(lk.cpu().numpy(), oracle.budget_fixed(3, L, s))
+
+
+def _gpu_scores(B, L, H, Hkv, seed, q=16):
+    x = make_inputs(B, L, H, Hkv, 128, torch.bfloat16, seed=seed)
+    Q, K = x["Q"].cuda(), x["K"].cuda()
+    s_h, s_l = tsa.tsa_score(Q, K, q)
+    return tsa.dims(Q, K), s_h
+
+
+@pytest.mark.parametrize("L", [5, 2 * 2048 + 1, 5000])
+@pytest.mark.parametrize("width", [1, 3, 7, 63, 255])
+def test_pool_matches_oracle(L, width):
+    dm, s_h = _gpu_scores(2, L, 8, 2, seed=L + width)
+    raw = s_h.cpu().numpy()
+    for kind in (tsa.POOL_MAX, tsa.POOL_MEAN):
+        p, sl = tsa.tsa_pool_scores(dm, s_h, kind, width)
+        got = p.cpu().numpy().astype(np.float64)
+        ref_p, ref_sl = oracle.pool(raw, kind, width)
+        if kind == tsa.POOL_MAX:
+            np.testing.assert_array_equal(got, ref_p)
+        else:
+            rel = np.abs(got - ref_p) / np.maximum(ref_p, 1e-30)
+            assert rel.max() <= (width + 1) * 2.0 ** -23, rel.max()
+        assert_scores_close(sl.cpu().numpy(), ref_sl, "pooled s_l")
+
+
+def test_pool_rejects_bad_arguments_before_launch():
+    dm, s_h = _gpu_scores(1, 64, 4, 4, seed=3)
+    n0 = tsa.kernel_launches()
+    for kind, width, code in ((0, 3, 1), (3, 3, 1), (1, 4, 1), (2, 257, 3)):
+        with pytest.raises(tsa.TSAError) as e:
+            tsa.tsa_pool_scores(dm, s_h, kind, width)
+        assert e.value.status == code
+    with pytest.raises(tsa.TSAError):
+        tsa.tsa_pool_scores(dm, s_h, 1, 3, s_h_out=s_h)   # output overlaps input
+    assert tsa.kernel_launches() == n0
+
+
+def _check_y(x, idx, lk, Y):
+    """Y against the oracle's attention on these indices (all heads)."""
+    Q, K, V, X = x["Q"], x["K"], x["V"], x["X"]
+    dt, dd, H = Q.dtype, Q.shape[3], Q.shape[2]
+    Oh = oracle.attend(Q, K, V, idx, lk)
+    _, Y_ref = oracle.decompress_residual(Oh, idx, lk, X)
+    Yg = Y.double().numpy()
+    Xd = X.double().numpy()
+    for b in range(Q.shape[0]):
+        for h in range(H):
+            seg = slice(h * dd, (h + 1) * dd)
+            kept, rest = idx[b, h, :lk[b]], idx[b, h, lk[b]:]
+            np.testing.assert_array_equal(Yg[b, rest, seg], Xd[b, rest, seg])
+            if len(kept):
+                diff = np.abs(Yg[b, kept, seg] - Y_ref[b, kept, seg])
+                bound = ATOL[dt] + HALF_ULP[dt] * np.abs(Y_ref[b, kept, seg])
+                assert np.all(diff <= bound), "Y max excess %.3g" % (diff - bound).max()
+
+
+@pytest.mark.parametrize("variant", ["pool_max", "pool_mean", "fixed", "fixed_pool"])
+def test_layer_ex_matches_oracle(variant):
+    B, L, H, Hkv, q, tau = 2, 1000, 8, 2, 16, 0.02
+    x = make_inputs(B, L, H, Hkv, 128, torch.bfloat16, seed=41)
+    d = {k: v.cuda() for k, v in x.items()}
+    pool = {"pool_max": tsa.POOL_MAX, "pool_mean": tsa.POOL_MEAN, "fixed": tsa.POOL_NONE,
+            "fixed_pool": tsa.POOL_MAX}[variant]
+    sparsity = 0.3 if variant.startswith("fixed") else None
+    width = 7 if pool else 1
+    s_h = torch.empty(B, H, L, device="cuda")
+    s_l = torch.empty(B, L, device="cuda")
+    Lk = torch.empty(B, dtype=torch.int32, device="cuda")
+    idx = torch.empty(B, H, L, dtype=torch.int32, device="cuda")
+    Y = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=q, tau=tau, s_h=s_h, s_l=s_l,
+                      Lkeep=Lk, idx=idx, sparsity=sparsity, pool=pool, pool_width=width)
+    raw, _ = tsa.tsa_score(d["Q"], d["K"], q)
+    torch.cuda.synchronize()
+    raw = raw.cpu().numpy()
+    g_sh, g_sl = s_h.cpu().numpy(), s_l.cpu().numpy()
+    # the scores selection used: the pooled GPU scores (pooling checked above), else raw
+    if pool:
+        ref_p, ref_sl = oracle.pool(raw, pool, width)
+        if pool == tsa.POOL_MAX:
+            np.testing.assert_array_equal(g_sh.astype(np.float64), ref_p)
+        else:
+            assert np.max(np.abs(g_sh - ref_p) / np.maximum(ref_p, 1e-30)) <= 8 * 2.0 ** -23
+        assert_scores_close(g_sl, ref_sl, "layer s_l")
+    else:
+        np.testing.assert_array_equal(g_sh, raw)
+    lk = (oracle.budget_fixed(B, L, sparsity) if sparsity is not None
+          else oracle.budget(g_sl, tau)[0])
+    np.testing.assert_array_equal(Lk.cpu().numpy(), lk)
+    ref_idx = oracle.select(g_sh, lk)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    _check_y(x, ref_idx, lk, Y.cpu())

@@ -17,6 +17,8 @@ cudaError_t launch_score_simt(const tsa_dims &, const void *, const void *, int,
                               const WsLayout &, char *, cudaStream_t);
 cudaError_t launch_score_tc(const tsa_dims &, const void *, const void *, int, float, float *,
                             const WsLayout &, char *, cudaStream_t, uint32_t);
+cudaError_t launch_fill_lkeep(int, int32_t, int32_t *, cudaStream_t);
+cudaError_t launch_pool(const tsa_dims &, const float *, int, int, float *, cudaStream_t);
 cudaError_t launch_norm(const tsa_dims &, const float *, float *, const WsLayout &, char *,
                         cudaStream_t);
 cudaError_t launch_budget(const tsa_dims &, const float *, double, int32_t *, char *,
@@ -126,7 +128,7 @@ WsLayout ws_layout(const tsa_dims &dm, int q) {
 }
 
 struct LayerLayout {
-    size_t s_h, s_l, lkeep, idx, qh, kh, vh, oh, total;
+    size_t s_h, s_hp, s_l, lkeep, idx, qh, kh, vh, oh, total;
 };
 
 static LayerLayout layer_layout(const tsa_dims &dm, int q) {
@@ -134,6 +136,7 @@ static LayerLayout layer_layout(const tsa_dims &dm, int q) {
     size_t off = ws_layout(dm, q).total;
     const size_t BHL = (size_t)dm.B * dm.H * dm.L;
     y.s_h = off; off = align256(off + 4 * BHL);
+    y.s_hp = off; off = align256(off + 4 * BHL);  // pooled head scores (score variant)
     y.s_l = off; off = align256(off + 4 * (size_t)dm.B * dm.L);
     y.lkeep = off; off = align256(off + 4 * (size_t)dm.B);
     y.idx = off; off = align256(off + 4 * BHL);
@@ -279,15 +282,67 @@ tsa_status tsa_scatter_residual(const tsa_dims *dims, const void *Oh, const int3
                        "tsa_scatter_residual");
 }
 
-tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const void *V,
-                     const void *X, void *Y, int32_t is_sparse, int32_t q, double tau,
-                     float scale, float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
-                     int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
-                     void *const *stage_events) {
+static tsa_status check_pool(int32_t kind, int32_t width) {
+    if (kind != TSA_POOL_MAX && kind != TSA_POOL_MEAN)
+        return fail(TSA_ERR_INVALID_ARG, "pool kind must be TSA_POOL_MAX or TSA_POOL_MEAN");
+    if (width < 1 || (width & 1) == 0) return fail(TSA_ERR_INVALID_ARG, "pool width must be odd");
+    if (width > 255) return fail(TSA_ERR_UNSUPPORTED, "pool width above 255");
+    return TSA_OK;
+}
+
+static tsa_status check_sparsity(double s) {
+    if (!(s >= 0.0 && s <= 1.0)) return fail(TSA_ERR_INVALID_ARG, "sparsity must be in [0, 1]");
+    return TSA_OK;
+}
+
+// L' of the fixed-ratio budget: L - floor(s * L), the product in double.
+static int32_t fixed_keep(int L, double s) { return L - (int32_t)floor(s * (double)L); }
+
+tsa_status tsa_budget_fixed(const tsa_dims *dims, double sparsity, int32_t *Lkeep,
+                            void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_sparsity(sparsity));
+    TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    return cuda_status(launch_fill_lkeep(dims->B, fixed_keep(dims->L, sparsity), Lkeep,
+                                         (cudaStream_t)stream),
+                       "tsa_budget_fixed");
+}
+
+tsa_status tsa_pool_scores(const tsa_dims *dims, const float *s_h, int32_t kind, int32_t width,
+                           float *s_h_out, float *s_l_out, void *ws, size_t ws_bytes,
+                           void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_pool(kind, width));
+    TSA_TRY(check_ptr(s_h, "s_h"));
+    TSA_TRY(check_ptr(s_h_out, "s_h_out"));
+    TSA_TRY(check_ptr(s_l_out, "s_l_out"));
+    const size_t bytes = (size_t)4 * dims->B * dims->H * dims->L;
+    const char *a = (const char *)s_h, *o = (const char *)s_h_out;
+    if (a < o + bytes && o < a + bytes) return fail(TSA_ERR_INVALID_ARG, "s_h_out overlaps s_h");
+    const WsLayout w = ws_layout(*dims, 1);
+    TSA_TRY(check_ws(ws, ws_bytes, w.total));
+    cudaStream_t st = (cudaStream_t)stream;
+    TSA_TRY(cuda_status(launch_pool(*dims, s_h, kind, width, s_h_out, st), "tsa_pool_scores"));
+    return cuda_status(launch_norm(*dims, s_h_out, s_l_out, w, (char *)ws, st),
+                       "tsa_pool_scores (normalise)");
+}
+
+static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K, const void *V,
+                             const void *X, void *Y, int32_t is_sparse, int32_t q,
+                             const tsa_layer_opts &o, float scale, float *s_h_out,
+                             float *s_l_out, int32_t *Lkeep_out, int32_t *idx_out, void *ws,
+                             size_t ws_bytes, void *stream, void *const *stage_events) {
     TSA_TRY(check_dims(dims));
     TSA_TRY(check_q(dims, q));
     TSA_TRY(check_scale(scale));
-    if (!(tau >= 0.0 && tau < 1.0)) return fail(TSA_ERR_INVALID_ARG, "tau must be in [0, 1)");
+    if (o.budget == TSA_BUDGET_COVERAGE) {
+        if (!(o.tau >= 0.0 && o.tau < 1.0)) return fail(TSA_ERR_INVALID_ARG, "tau must be in [0, 1)");
+    } else if (o.budget == TSA_BUDGET_FIXED) {
+        TSA_TRY(check_sparsity(o.sparsity));
+    } else {
+        return fail(TSA_ERR_INVALID_ARG, "unknown budget kind");
+    }
+    if (o.pool != TSA_POOL_NONE) TSA_TRY(check_pool(o.pool, o.pool_width));
     TSA_TRY(check_ptr(Q, "Q"));
     TSA_TRY(check_ptr(K, "K"));
     TSA_TRY(check_ptr(V, "V"));
@@ -305,7 +360,10 @@ tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const v
         if (!stage_events) return TSA_OK;
         return cuda_status(cudaEventRecord((cudaEvent_t)stage_events[i], st), "event record");
     };
-    float *s_h = s_h_out ? s_h_out : (float *)(w + y.s_h);
+    const bool pooled = o.pool != TSA_POOL_NONE;
+    // Scores used by budget and selection: the raw ones, or the pooled ones.
+    float *s_raw = (s_h_out && !pooled) ? s_h_out : (float *)(w + y.s_h);
+    float *s_h = !pooled ? s_raw : (s_h_out ? s_h_out : (float *)(w + y.s_hp));
     float *s_l = s_l_out ? s_l_out : (float *)(w + y.s_l);
     int32_t *Lk = Lkeep_out ? Lkeep_out : (int32_t *)(w + y.lkeep);
     int32_t *idx = idx_out ? idx_out : (int32_t *)(w + y.idx);
@@ -318,9 +376,19 @@ tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const v
         return rec(6);
     }
     TSA_TRY(rec(0));
-    TSA_TRY(do_score(dm, Q, K, q, scale, s_h, s_l, w, st));
+    TSA_TRY(do_score(dm, Q, K, q, scale, s_raw, s_l, w, st));
+    if (pooled) {
+        TSA_TRY(cuda_status(launch_pool(dm, s_raw, o.pool, o.pool_width, s_h, st),
+                            "tsa_layer pool"));
+        TSA_TRY(cuda_status(launch_norm(dm, s_h, s_l, ws_layout(dm, q), w, st),
+                            "tsa_layer pool (normalise)"));
+    }
     TSA_TRY(rec(1));
-    TSA_TRY(cuda_status(launch_budget(dm, s_l, tau, Lk, w, st), "tsa_layer budget"));
+    if (o.budget == TSA_BUDGET_COVERAGE)
+        TSA_TRY(cuda_status(launch_budget(dm, s_l, o.tau, Lk, w, st), "tsa_layer budget"));
+    else
+        TSA_TRY(cuda_status(launch_fill_lkeep(dm.B, fixed_keep(dm.L, o.sparsity), Lk, st),
+                            "tsa_layer budget"));
     TSA_TRY(rec(2));
     TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, w, st), "tsa_layer select"));
     TSA_TRY(rec(3));
@@ -331,6 +399,27 @@ tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const v
     TSA_TRY(rec(5));
     TSA_TRY(cuda_status(launch_scatter(dm, Oh, idx, Lk, X, Y, st), "tsa_layer scatter"));
     return rec(6);
+}
+
+tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const void *V,
+                     const void *X, void *Y, int32_t is_sparse, int32_t q, double tau,
+                     float scale, float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
+                     int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
+                     void *const *stage_events) {
+    tsa_layer_opts o{TSA_BUDGET_COVERAGE, tau, 0.0, TSA_POOL_NONE, 1};
+    return layer_impl(dims, Q, K, V, X, Y, is_sparse, q, o, scale, s_h_out, s_l_out, Lkeep_out,
+                      idx_out, ws, ws_bytes, stream, stage_events);
+}
+
+tsa_status tsa_layer_ex(const tsa_dims *dims, const void *Q, const void *K, const void *V,
+                        const void *X, void *Y, int32_t is_sparse, int32_t q,
+                        const tsa_layer_opts *opts, float scale, float *s_h_out,
+                        float *s_l_out, int32_t *Lkeep_out, int32_t *idx_out, void *ws,
+                        size_t ws_bytes, void *stream, void *const *stage_events) {
+    const tsa_layer_opts o = opts ? *opts
+                                  : tsa_layer_opts{TSA_BUDGET_COVERAGE, 0.005, 0.0, TSA_POOL_NONE, 1};
+    return layer_impl(dims, Q, K, V, X, Y, is_sparse, q, o, scale, s_h_out, s_l_out, Lkeep_out,
+                      idx_out, ws, ws_bytes, stream, stage_events);
 }
 
 tsa_status tsa_get_device_status(void *ws, void *stream) {

@@ -24,7 +24,9 @@ EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_b
            "tsa_select", "tsa_gather_qkv", "tsa_attn", "tsa_scatter_residual", "tsa_layer",
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
            "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall",
-           "tsa_kernel_launches")
+           "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex")
+POOL_NONE, POOL_MAX, POOL_MEAN = 0, 1, 2
+BUDGET_COVERAGE, BUDGET_FIXED = 0, 1
 
 
 class TSAError(RuntimeError):
@@ -36,6 +38,13 @@ class TSAError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class LayerOpts(ctypes.Structure):
+    """tsa_layer_opts of include/tsa.h."""
+    _fields_ = [("budget", ctypes.c_int32), ("tau", ctypes.c_double),
+                ("sparsity", ctypes.c_double), ("pool", ctypes.c_int32),
+                ("pool_width", ctypes.c_int32)]
 
 
 def lib():
@@ -65,6 +74,10 @@ def lib():
             "tsa_status_string": (ctypes.c_char_p, [I32]),
             "tsa_last_error": (ctypes.c_char_p, []),
             "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
+            "tsa_budget_fixed": (I32, [DP, D, P, P]),
+            "tsa_pool_scores": (I32, [DP, P, I32, I32, P, P, P, SZ, P]),
+            "tsa_layer_ex": (I32, [DP, P, P, P, P, P, I32, I32, ctypes.POINTER(LayerOpts), F,
+                                   P, P, P, P, P, SZ, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -212,10 +225,37 @@ def tsa_scatter_residual(dm: Dims, Oh, idx, Lkeep, X, Y=None, stream=None):
     return Y
 
 
+def tsa_budget_fixed(dm: Dims, sparsity: float, Lkeep=None, device=None, stream=None):
+    """Fixed-ratio budget: Lkeep[b] = L - floor(sparsity * L)."""
+    if Lkeep is None:
+        Lkeep = torch.empty(dm.B, dtype=torch.int32, device=device or "cuda")
+    _need_cuda(Lkeep)
+    _check(lib().tsa_budget_fixed(ctypes.byref(dm), float(sparsity), _p(Lkeep), _stream(stream)))
+    return Lkeep
+
+
+def tsa_pool_scores(dm: Dims, s_h, kind: int, width: int, s_h_out=None, s_l_out=None, ws=None,
+                    stream=None):
+    """Token-axis max / mean pooling of s_h [B, H, L]; returns (pooled s_h, s_l)."""
+    _need_cuda(s_h)
+    if s_h_out is None:
+        s_h_out = torch.empty_like(s_h)
+    if s_l_out is None:
+        s_l_out = torch.empty(dm.B, dm.L, dtype=torch.float32, device=s_h.device)
+    if ws is None:
+        ws = workspace(dm, 1, device=s_h.device)
+    _check(lib().tsa_pool_scores(ctypes.byref(dm), _p(s_h), int(kind), int(width), _p(s_h_out),
+                                 _p(s_l_out), _p(ws), ws.numel(), _stream(stream)))
+    return s_h_out, s_l_out
+
+
 def tsa_layer(Q, K, V, X, Y=None, is_sparse: bool = True, q: int = 16, tau: float = 0.005,
               scale: float | None = None, s_h=None, s_l=None, Lkeep=None, idx=None, ws=None,
-              stream=None, stage_events=None):
-    """One Token Sparse Attention layer: returns Y = X + Decompress(Ô) (or the dense layer)."""
+              stream=None, stage_events=None, sparsity: float | None = None,
+              pool: int = POOL_NONE, pool_width: int = 1):
+    """One Token Sparse Attention layer: returns Y = X + Decompress(Ô) (or the dense layer).
+    sparsity (fixed-ratio budget instead of tau) and pool / pool_width (pooled head
+    scores) select the variants of tsa_layer_ex."""
     dm = dims(Q, K)
     _need_cuda(Q, K, V, X, Y, s_h, s_l, Lkeep, idx)
     if Y is None:
@@ -225,10 +265,17 @@ def tsa_layer(Q, K, V, X, Y=None, is_sparse: bool = True, q: int = 16, tau: floa
     ev = None
     if stage_events is not None:
         ev = (ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
-    _check(lib().tsa_layer(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y), int(is_sparse),
-                           q, float(tau), default_scale(dm.d) if scale is None else scale,
-                           _p(s_h), _p(s_l), _p(Lkeep), _p(idx), _p(ws), ws.numel(),
-                           _stream(stream), ev))
+    sc = default_scale(dm.d) if scale is None else scale
+    if sparsity is None and pool == POOL_NONE:
+        _check(lib().tsa_layer(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y),
+                               int(is_sparse), q, float(tau), sc, _p(s_h), _p(s_l), _p(Lkeep),
+                               _p(idx), _p(ws), ws.numel(), _stream(stream), ev))
+        return Y
+    o = LayerOpts(BUDGET_COVERAGE if sparsity is None else BUDGET_FIXED, float(tau),
+                  0.0 if sparsity is None else float(sparsity), int(pool), int(pool_width))
+    _check(lib().tsa_layer_ex(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y),
+                              int(is_sparse), q, ctypes.byref(o), sc, _p(s_h), _p(s_l),
+                              _p(Lkeep), _p(idx), _p(ws), ws.numel(), _stream(stream), ev))
     return Y
 
 
