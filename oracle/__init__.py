@@ -49,8 +49,11 @@ def _load():
         lib.orc_decompress_residual.argtypes = [I, I, I, I, I, P, P, P, P, P, P]
         lib.orc_budget_fixed.argtypes = [I, I, D, P]
         lib.orc_pool.argtypes = [I, I, I, P, I, I, P, P]
+        lib.orc_drift.argtypes = [I, L, I, I, P, D, P]
+        lib.orc_drift_mask.argtypes = [I, P, D, P]
         for f in ("orc_score", "orc_budget", "orc_select", "orc_attend_rows",
-                  "orc_decompress_residual", "orc_budget_fixed", "orc_pool"):
+                  "orc_decompress_residual", "orc_budget_fixed", "orc_pool", "orc_drift",
+                  "orc_drift_mask"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -147,6 +150,28 @@ def pool(s_h, kind: int, width: int):
     if rc:
         raise ValueError("orc_pool rejected its arguments (%d)" % rc)
     return out, sl
+
+
+def drift(h, eps: float = 1e-6):
+    """Per-layer drift R [N] (fp64) of hidden states h [N + 1, T, D] (fp32 or bf16)."""
+    a = _np(h)
+    N1, T, D = a.shape
+    a = np.ascontiguousarray(a)
+    R = np.zeros(N1 - 1, np.float64)
+    rc = _load().orc_drift(N1 - 1, T, D, _dtype_code(a), _ptr(a), float(eps), _ptr(R))
+    if rc:
+        raise ValueError("orc_drift rejected its arguments (%d)" % rc)
+    return R
+
+
+def drift_mask(R, delta: float = 0.5):
+    """Sparse-layer mask int32 [N]: 1 where rank(R_l) / N <= delta."""
+    r = np.ascontiguousarray(_np(R), dtype=np.float64)
+    mask = np.zeros(len(r), np.int32)
+    rc = _load().orc_drift_mask(len(r), _ptr(r), float(delta), _ptr(mask))
+    if rc:
+        raise ValueError("orc_drift_mask rejected its arguments (%d)" % rc)
+    return mask
 
 
 def select(s_h, Lkeep):

@@ -403,3 +403,44 @@ int orc_decompress_residual(int B, int L, int H, int d, int dtype,
     if (!O_dec) free(O);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Sparse-layer choice by inter-layer representation drift.  [notes] 关键设计 */
+/* 3 (R_l = E_t[ ||h_{l+1,t} - h_{l,t}||_2 / (||h_{l,t}||_2 + eps) ], rank,  */
+/* sparse layers = { l : R^_l <= delta }, delta = 0.5 by default); [blog] §2 */
+/* (only the layers in the lower 50% of the drift ranking, i.e. below the    */
+/* median, are made sparse).  Readings: R^_l = rank_l / N with rank_l the     */
+/* 1-based position in ascending R (ties: lower layer first); the mean runs  */
+/* over all T calibration tokens; eps is the caller's (the pages give none).  */
+/* h holds N + 1 states [N + 1, T, D]: h_0 the input of layer 0, h_{l+1} the  */
+/* output of layer l.                                                        */
+/* ------------------------------------------------------------------------ */
+int orc_drift(int N, long T, int D, int dtype, const void *h, double eps, double *R) {
+    if (N < 1 || T < 1 || D < 1 || !(eps >= 0.0)) return 1;
+    for (int l = 0; l < N; ++l) {
+        double acc = 0.0;
+        for (long t = 0; t < T; ++t) {
+            const size_t a = ((size_t)l * T + t) * D, b = ((size_t)(l + 1) * T + t) * D;
+            double dd = 0.0, hh = 0.0;
+            for (int c = 0; c < D; ++c) {
+                const double x = elem(h, dtype, a + c), y = elem(h, dtype, b + c);
+                dd += (y - x) * (y - x);
+                hh += x * x;
+            }
+            acc += sqrt(dd) / (sqrt(hh) + eps);
+        }
+        R[l] = acc / (double)T;
+    }
+    return 0;
+}
+
+int orc_drift_mask(int N, const double *R, double delta, int32_t *mask) {
+    if (N < 1 || !(delta >= 0.0 && delta <= 1.0)) return 1;
+    for (int l = 0; l < N; ++l) {
+        int rank = 1;
+        for (int m = 0; m < N; ++m)
+            if (R[m] < R[l] || (R[m] == R[l] && m < l)) ++rank;
+        mask[l] = ((double)rank / (double)N <= delta) ? 1 : 0;
+    }
+    return 0;
+}

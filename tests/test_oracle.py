@@ -393,3 +393,52 @@ def test_pool_rejects_bad_arguments():
     for kind, width in ((3, 3), (1, 2), (2, 0)):
         with pytest.raises(ValueError):
             oracle.pool(s, kind, width)
+
+
+# ---------------------------------------------------------------- drift pass
+def test_drift_identical_states_are_zero_and_mask_takes_lowest_indices():
+    h = np.tile(np.random.default_rng(0).standard_normal((1, 6, 16)).astype(np.float32), (9, 1, 1))
+    R = oracle.drift(h)
+    np.testing.assert_array_equal(R, 0.0)
+    np.testing.assert_array_equal(oracle.drift_mask(R, 0.5), [1, 1, 1, 1, 0, 0, 0, 0])
+
+
+def test_drift_of_scaled_states_is_the_scale_step():
+    rng = np.random.default_rng(1)
+    c = [2.0, 0.5, 4.0, 1.0, 0.25]
+    h = [rng.standard_normal((7, 32)).astype(np.float32)]
+    for k in c:
+        h.append((h[-1] * np.float32(k)).astype(np.float32))   # exact: powers of two
+    R = oracle.drift(np.stack(h), eps=0.0)
+    np.testing.assert_allclose(R, [abs(k - 1) for k in c], rtol=1e-12)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_drift_matches_numpy_norms(dtype):
+    h = torch.randn(5, 11, 64).to(dtype)
+    eps = 1e-3
+    R = oracle.drift(h, eps=eps)
+    hd = h.double().numpy()
+    want = [np.mean(np.linalg.norm(hd[l + 1] - hd[l], axis=1) / (np.linalg.norm(hd[l], axis=1) + eps))
+            for l in range(4)]
+    np.testing.assert_allclose(R, want, rtol=1e-12)
+
+
+@pytest.mark.parametrize("N,delta", [(32, 0.5), (5, 0.5), (7, 0.3), (4, 1.0), (4, 0.0)])
+def test_drift_mask_brute_force(N, delta):
+    rng = np.random.default_rng(N)
+    R = rng.integers(0, 4, N).astype(np.float64) / 4        # ties on purpose
+    order = sorted(range(N), key=lambda l: (R[l], l))
+    want = np.zeros(N, np.int32)
+    for rank, l in enumerate(order, start=1):
+        want[l] = Fraction(rank, N) <= Fraction(delta)
+    np.testing.assert_array_equal(oracle.drift_mask(R, delta), want)
+    if N == 32 and delta == 0.5:
+        assert want.sum() == 16                               # half the layers sparse
+
+
+def test_drift_rejects_bad_arguments():
+    with pytest.raises(ValueError):
+        oracle.drift(np.zeros((1, 3, 4), np.float32))         # needs two states
+    with pytest.raises(ValueError):
+        oracle.drift_mask(np.zeros(3), 1.5)
