@@ -4,8 +4,10 @@
  * The method is from "Token Sparse Attention: Efficient Long-Context Inference with
  * Interleaved Token Selection".  Page citations below:
  *   [notes] the papernotes.org notes on that paper (方法详解 › 整体框架; 关键设计 1
- *           Compress-then-Decompress; 关键设计 2 Dynamic Token Coverage);
- *   [blog]  the bxzpzcl.cn post (§1.1 核心算法实现细节; §2.1 重要性评估机制);
+ *           Compress-then-Decompress; 关键设计 2 Dynamic Token Coverage; 关键设计 3
+ *           Inter-Layer Representation Drift; 消融实验 ablations);
+ *   [blog]  the bxzpzcl.cn post (§1.1 核心算法实现细节; §2 稀疏层选择 by drift;
+ *           §2.1 重要性评估机制);
  *   [gist]  the gist.science summary (§2 Methodology: Core Architecture; Dynamic
  *           Token Coverage).
  *
@@ -212,6 +214,27 @@ TSA_API tsa_status tsa_layer_ex(const tsa_dims *dims, const void *Q, const void 
                                 float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
                                 int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
                                 void *const *stage_events);
+
+/* ---- Choice of the sparse layers ([notes] 关键设计 3) ------------------------------ */
+
+/* Bytes of workspace tsa_drift needs (0 on invalid arguments). */
+TSA_API size_t tsa_drift_workspace_size(int32_t n_layers, int64_t tokens);
+
+/* Inter-layer representation drift on calibration hidden states and the sparse-layer
+ * mask ([notes] 关键设计 3; [blog] §2):
+ *   R[l] = mean over t of ||h[l+1,t] - h[l,t]||_2 / (||h[l,t]||_2 + eps),
+ *   mask[l] = 1 iff rank_l / n_layers <= delta, rank_l the 1-based position of R[l] in
+ *   ascending order (ties: lower layer first); delta = 0.5 makes the half of the layers
+ *   with the smallest drift sparse.
+ * h: [n_layers + 1, tokens, d_model] contiguous, dtype TSA_BF16 or TSA_F32 (h[0] the
+ * input of layer 0, h[l+1] the output of layer l), 16-byte aligned.  Norms are summed in
+ * fp32 per token, the token mean in fp64, in a fixed order (deterministic).  R [n_layers]
+ * fp64 and mask [n_layers] int32 are device outputs.  1 <= n_layers <= 512;
+ * d_model * element size a multiple of 16 bytes; eps >= 0; delta in [0, 1].
+ * ws: tsa_drift_workspace_size() bytes, 256-byte aligned. */
+TSA_API tsa_status tsa_drift(int32_t n_layers, int64_t tokens, int32_t d_model, int32_t dtype,
+                             const void *h, double eps, double delta, double *R, int32_t *mask,
+                             void *ws, size_t ws_bytes, void *stream);
 
 /* Scoring for callers that cannot allocate device memory when they call in, such as an
  * engine whose device memory is fully planned up front by its own allocator, or a host

@@ -140,6 +140,20 @@ def test_variant_validation():
     assert tsa.workspace_size(dm, 16, layer=True) >= 2 * 4 * 32 * 4096 + 4 * 32 * 4096 * 128 * 2
 
 
+def test_drift_validation():
+    L = tsa.lib()
+    n0 = tsa.kernel_launches()
+    assert L.tsa_drift_workspace_size(0, 10) == 0 and L.tsa_drift_workspace_size(513, 10) == 0
+    assert L.tsa_drift_workspace_size(32, 4096) >= 256 + 64 * 32 * 8
+    dr = lambda N=4, T=100, D=256, dt=tsa.TSA_BF16, h=FAKE, eps=1e-6, delta=0.5, wsb=1 << 30: \
+        L.tsa_drift(N, T, D, dt, P(h), eps, delta, P(FAKE), P(FAKE), P(FAKE * 16), wsb, None)
+    assert dr(N=0) == 1 and dr(N=513) == 1 and dr(T=0) == 1
+    assert dr(D=4) == 3 and dr(dt=7) == 3                 # 8 bytes per row, unknown dtype
+    assert dr(eps=-1.0) == 1 and dr(delta=1.5) == 1 and dr(eps=float("nan")) == 1
+    assert dr(h=0) == 1 and dr(h=FAKE + 4) == 2 and dr(wsb=16) == 4
+    assert tsa.kernel_launches() == n0
+
+
 def test_failed_validation_launches_nothing():
     n0 = tsa.kernel_launches()
     dm = _d()

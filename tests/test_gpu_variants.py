@@ -119,3 +119,46 @@ def test_layer_ex_matches_oracle(variant):
     ref_idx = oracle.select(g_sh, lk)
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
     _check_y(x, ref_idx, lk, Y.cpu())
+
+
+# ---------------------------------------------------------------- drift pass
+def _drift_check(h, eps=1e-6, delta=0.5):
+    R, mask = tsa.tsa_drift(h.cuda(), eps=eps, delta=delta)
+    R, mask = R.cpu().numpy(), mask.cpu().numpy()
+    ref = oracle.drift(h, eps=eps)
+    rel = np.abs(R - ref) / np.maximum(np.abs(ref), 1e-30)
+    assert rel.max() <= 1e-5, rel.max()
+    np.testing.assert_array_equal(mask, oracle.drift_mask(R, delta))   # decision on GPU's R
+    return R, mask
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T", [1, 100, 1000])
+def test_drift_matches_oracle(dtype, T):
+    g = torch.Generator().manual_seed(T)
+    N, D = 6, 256
+    steps = torch.rand(N, generator=g) * 0.5                  # a different drift per layer
+    h = [torch.randn(T, D, generator=g)]
+    for l in range(N):
+        h.append(h[-1] + steps[l] * torch.randn(T, D, generator=g))
+    _drift_check(torch.stack(h).to(dtype).contiguous(), delta=0.5)
+
+
+def test_drift_identical_states_and_determinism():
+    h = torch.randn(1, 300, 512).to(torch.bfloat16).expand(9, 300, 512).contiguous()
+    R, mask = _drift_check(h)
+    assert np.all(R == 0) and list(mask) == [1, 1, 1, 1, 0, 0, 0, 0]
+    x = torch.randn(33, 257, 1024, dtype=torch.bfloat16).cuda()
+    a = tsa.tsa_drift(x)
+    b = tsa.tsa_drift(x)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_drift_llama_width_32_layers():
+    g = torch.Generator().manual_seed(5)
+    N, T, D = 32, 512, 4096
+    h = [torch.randn(T, D, generator=g)]
+    for l in range(N):
+        h.append(h[-1] * 0.9 + (0.05 + 0.01 * (l % 7)) * torch.randn(T, D, generator=g))
+    R, mask = _drift_check(torch.stack(h).to(torch.bfloat16).contiguous())
+    assert mask.sum() == 16

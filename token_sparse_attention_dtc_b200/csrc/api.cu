@@ -18,6 +18,9 @@ cudaError_t launch_score_simt(const tsa_dims &, const void *, const void *, int,
 cudaError_t launch_score_tc(const tsa_dims &, const void *, const void *, int, float, float *,
                             const WsLayout &, char *, cudaStream_t, uint32_t);
 cudaError_t launch_fill_lkeep(int, int32_t, int32_t *, cudaStream_t);
+size_t drift_workspace_bytes(int, long long);
+cudaError_t launch_drift(int, long long, int, int, const void *, double, double, double *,
+                         int32_t *, char *, cudaStream_t);
 cudaError_t launch_pool(const tsa_dims &, const float *, int, int, float *, cudaStream_t);
 cudaError_t launch_norm(const tsa_dims &, const float *, float *, const WsLayout &, char *,
                         cudaStream_t);
@@ -420,6 +423,37 @@ tsa_status tsa_layer_ex(const tsa_dims *dims, const void *Q, const void *K, cons
                                   : tsa_layer_opts{TSA_BUDGET_COVERAGE, 0.005, 0.0, TSA_POOL_NONE, 1};
     return layer_impl(dims, Q, K, V, X, Y, is_sparse, q, o, scale, s_h_out, s_l_out, Lkeep_out,
                       idx_out, ws, ws_bytes, stream, stage_events);
+}
+
+static tsa_status check_drift(int32_t n_layers, int64_t tokens, int32_t d_model, int32_t dtype) {
+    if (n_layers < 1 || n_layers > 512)
+        return fail(TSA_ERR_INVALID_ARG, "n_layers must be in [1, 512]");
+    if (tokens < 1 || tokens > ((int64_t)1 << 36)) return fail(TSA_ERR_INVALID_ARG, "bad token count");
+    if (dtype != TSA_F32 && dtype != TSA_BF16) return fail(TSA_ERR_UNSUPPORTED, "dtype");
+    const int esz = dtype == TSA_F32 ? 4 : 2;
+    if (d_model < 1 || d_model > 65536 || (d_model * esz) % 16)
+        return fail(TSA_ERR_UNSUPPORTED, "d_model * element size must be a multiple of 16 bytes");
+    return TSA_OK;
+}
+
+size_t tsa_drift_workspace_size(int32_t n_layers, int64_t tokens) {
+    if (n_layers < 1 || n_layers > 512 || tokens < 1 || tokens > ((int64_t)1 << 36)) return 0;
+    return drift_workspace_bytes(n_layers, tokens);
+}
+
+tsa_status tsa_drift(int32_t n_layers, int64_t tokens, int32_t d_model, int32_t dtype,
+                     const void *h, double eps, double delta, double *R, int32_t *mask, void *ws,
+                     size_t ws_bytes, void *stream) {
+    TSA_TRY(check_drift(n_layers, tokens, d_model, dtype));
+    if (!(eps >= 0.0 && eps < 1e30)) return fail(TSA_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    if (!(delta >= 0.0 && delta <= 1.0)) return fail(TSA_ERR_INVALID_ARG, "delta must be in [0, 1]");
+    TSA_TRY(check_ptr(h, "h"));
+    TSA_TRY(check_ptr(R, "R"));
+    TSA_TRY(check_ptr(mask, "mask"));
+    TSA_TRY(check_ws(ws, ws_bytes, drift_workspace_bytes(n_layers, tokens)));
+    return cuda_status(launch_drift(n_layers, tokens, d_model, dtype, h, eps, delta, R, mask,
+                                    (char *)ws, (cudaStream_t)stream),
+                       "tsa_drift");
 }
 
 tsa_status tsa_get_device_status(void *ws, void *stream) {

@@ -24,7 +24,8 @@ EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_b
            "tsa_select", "tsa_gather_qkv", "tsa_attn", "tsa_scatter_residual", "tsa_layer",
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
            "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall",
-           "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex")
+           "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex",
+           "tsa_drift_workspace_size", "tsa_drift")
 POOL_NONE, POOL_MAX, POOL_MEAN = 0, 1, 2
 BUDGET_COVERAGE, BUDGET_FIXED = 0, 1
 
@@ -75,6 +76,8 @@ def lib():
             "tsa_last_error": (ctypes.c_char_p, []),
             "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
             "tsa_budget_fixed": (I32, [DP, D, P, P]),
+            "tsa_drift_workspace_size": (SZ, [I32, ctypes.c_int64]),
+            "tsa_drift": (I32, [I32, ctypes.c_int64, I32, I32, P, D, D, P, P, P, SZ, P]),
             "tsa_pool_scores": (I32, [DP, P, I32, I32, P, P, P, SZ, P]),
             "tsa_layer_ex": (I32, [DP, P, P, P, P, P, I32, I32, ctypes.POINTER(LayerOpts), F,
                                    P, P, P, P, P, SZ, P, P]),
@@ -223,6 +226,24 @@ def tsa_scatter_residual(dm: Dims, Oh, idx, Lkeep, X, Y=None, stream=None):
     _check(lib().tsa_scatter_residual(ctypes.byref(dm), _p(Oh), _p(idx), _p(Lkeep), _p(X),
                                       _p(Y), _stream(stream)))
     return Y
+
+
+def tsa_drift(h, eps: float = 1e-6, delta: float = 0.5, ws=None, stream=None):
+    """Drift R [N] (fp64) and sparse-layer mask [N] (int32) of hidden states h
+    [N + 1, T, D] (bf16 or fp32, on the GPU)."""
+    _need_cuda(h)
+    if h.dim() != 3 or not h.is_contiguous():
+        raise ValueError("h must be a contiguous [N + 1, T, D] tensor")
+    N, T, D = h.shape[0] - 1, h.shape[1], h.shape[2]
+    dt = TSA_BF16 if h.dtype == torch.bfloat16 else TSA_F32
+    R = torch.empty(max(N, 0), dtype=torch.float64, device=h.device)
+    mask = torch.empty(max(N, 0), dtype=torch.int32, device=h.device)
+    if ws is None:
+        n = lib().tsa_drift_workspace_size(N, T)
+        ws = torch.zeros(max(n, 256), dtype=torch.uint8, device=h.device)
+    _check(lib().tsa_drift(N, T, D, dt, _p(h), float(eps), float(delta), _p(R), _p(mask),
+                           _p(ws), ws.numel(), _stream(stream)))
+    return R, mask
 
 
 def tsa_budget_fixed(dm: Dims, sparsity: float, Lkeep=None, device=None, stream=None):
