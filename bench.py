@@ -15,6 +15,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -26,6 +27,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "token-sparse attn layer ms @128K Llama-8B shape; TFLOP/s & % roofline"
 STAGES = ("score", "budget", "select", "gather", "attn", "scatter")
+# fractions of the tokens pruned at 128K in the pages' own runs (L' = 0.456 L and 0.326 L)
+PAGES_SPARSITY = (0.544, 0.674)
 
 
 def _peaks():
@@ -341,6 +344,38 @@ def run_ours(args, w, L, rank, world, local_rank):
                  "attn_frac_of_sustained": dflops / (dattn * 1e-3) / 1e12 / peaks["bf16_sus"],
                  "speedup_sparse_vs_dense_layer": dms / ms_step}
 
+    # the whole layer at the pages' sparsities (54.4% and 67.4% of the tokens pruned at
+    # 128K), through the fixed-ratio budget on the same synthetic inputs
+    pages = None
+    if not args.no_pages_sparsity:
+        pages = []
+        for sp in PAGES_SPARSITY:
+            lk_p = L - int(math.floor(sp * L))
+            for _ in range(2):
+                tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, ws=ws, sparsity=sp)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+            for e in ev:
+                e.record(st)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            sync_all()
+            a.record(st)
+            npg = 2
+            for _ in range(npg):
+                tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, ws=ws, sparsity=sp,
+                              stage_events=ev)
+            b.record(st)
+            sync_all()
+            pms = job_max(a.elapsed_time(b) / npg, world, dev)
+            pattn = ev[4].elapsed_time(ev[5])
+            pfl = 2.0 * w.H * w.d * lk_p * (lk_p + 1)
+            pages.append({"pruned": sp, "Lkeep": lk_p, "layer_ms": pms, "attn_ms": pattn,
+                          "attn_tflops": pfl / (pattn * 1e-3) / 1e12,
+                          "speedup_vs_dense_layer": (dense["layer_ms"] / pms) if dense else None,
+                          "data": "pages' sparsity, synthetic (fixed-ratio budget)"})
+        if tsa.tsa_get_device_status(ws) != 0:
+            raise RuntimeError("device error in the pages'-sparsity runs")
+
     # end to end through the public API with host buffers (copies inside the timed region)
     e2e = None
     if not args.no_e2e:
@@ -393,6 +428,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "layer_tflops": flops / (ms_step * 1e-3) / 1e12,
             "overhead_fraction": 1.0 - attn_ms / sum(stage_ms.values()),
             "dense": dense,
+            "pages_sparsity": pages,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
@@ -400,6 +436,149 @@ def run_ours(args, w, L, rank, world, local_rank):
             "peaks": peaks,
         }
         print(json.dumps(line), flush=True)
+
+
+def run_stack(args, L):
+    """32-layer stack (sparse and dense layers interleaved), one GPU.
+
+    Fresh synthetic Q/K/V per layer (seed*1000 + layer), the residual stream X updated in
+    place layer after layer.  The sparse set comes from the drift pass: an all-dense
+    calibration run records X_0..X_32, tsa_drift ranks the layers, delta = 0.5 makes half
+    of them sparse.  The stack is timed eagerly (one tsa_layer call per layer) and as a
+    captured CUDA graph replay, against the all-dense stack."""
+    import torch
+
+    from token_sparse_attention_dtc_b200 import tsa
+    from token_sparse_attention_dtc_b200.inputs import make_inputs
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    n_layers, H, Hkv, dd, q, tau = 32, 32, 8, 128, 16, 0.005
+    layers = []
+    for l in range(n_layers):
+        x = make_inputs(1, L, H, Hkv, dd, torch.bfloat16, seed=args.seed * 1000 + l)
+        layers.append({k: x[k].to(dev) for k in ("Q", "K", "V")})
+    X0 = make_inputs(1, L, H, Hkv, dd, torch.bfloat16, seed=args.seed * 1000 + 999)["X"].to(dev)
+    dm = tsa.dims(layers[0]["Q"], layers[0]["K"])
+    ws = tsa.workspace(dm, q, layer=True, device=dev)
+    X = X0.clone()
+    st = torch.cuda.current_stream(dev)
+
+    def stack(mask):
+        X.copy_(X0)
+        for l in range(n_layers):
+            c = layers[l]
+            tsa.tsa_layer(c["Q"], c["K"], c["V"], X, X, is_sparse=bool(mask[l]), q=q, tau=tau,
+                          ws=ws)
+
+    # calibration: all dense, keep every state for the drift pass
+    states = torch.empty(n_layers + 1, L, H * dd, dtype=torch.bfloat16, device=dev)
+    X.copy_(X0)
+    states[0].copy_(X0[0])
+    for l in range(n_layers):
+        c = layers[l]
+        tsa.tsa_layer(c["Q"], c["K"], c["V"], X, X, is_sparse=False, ws=ws)
+        states[l + 1].copy_(X[0])
+    R, mask_t = tsa.tsa_drift(states, eps=1e-6, delta=0.5)
+    mask = [int(v) for v in mask_t.cpu()]
+    del states
+
+    def timed(fn, n=3):
+        fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(n):
+            fn()
+        b.record(st)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    n0 = tsa.kernel_launches()
+    stack(mask)
+    launches = tsa.kernel_launches() - n0
+    eager_ms = timed(lambda: stack(mask))
+    dense_ms = timed(lambda: stack([0] * n_layers))
+    graph = {"replay_ms": None, "error": None}
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(st)
+        with torch.cuda.stream(side):
+            stack(mask)          # warm the launchers outside capture
+        st.wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            stack(mask)
+        graph["replay_ms"] = timed(g.replay)
+        Yg = X.clone()
+        stack(mask)
+        torch.cuda.synchronize()
+        graph["replay_equals_eager"] = bool(torch.equal(Yg, X))
+        del g
+    except Exception as e:  # capture is reported, not required
+        graph["error"] = str(e).splitlines()[0][:200]
+    if tsa.tsa_get_device_status(ws) != 0:
+        raise RuntimeError("device error in the stack run")
+    line = {
+        "metric": "32-layer stack ms (sparse set by drift, delta 0.5), Llama-8B heads",
+        "value": graph["replay_ms"] or eager_ms, "unit": "ms", "n_gpus": 1,
+        "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "stack32: B=1, L=%d, H=32, Hkv=8, d=128, bf16, q=16, "
+                               "tau=0.005, fresh Q/K/V per layer, X chained in place" % L},
+        "eager_ms": eager_ms, "graph": graph, "all_dense_ms": dense_ms,
+        "speedup_vs_all_dense": dense_ms / (graph["replay_ms"] or eager_ms),
+        "sparse_layers": [l for l in range(n_layers) if mask[l]],
+        "drift_R": [round(float(v), 6) for v in R.cpu()],
+        "gpu_launches_per_stack": launches,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_sweep(args):
+    """tau x q sweep on two 64K-token sequences (B = 2): one JSON line per setting."""
+    import torch
+
+    from token_sparse_attention_dtc_b200 import tsa
+    from token_sparse_attention_dtc_b200.inputs import WORKLOADS, make_workload
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    name = "llama8b_64k_b2"
+    x = make_workload(name, seed=args.seed)
+    d = {k: v.to(dev) for k, v in x.items()}
+    dm = tsa.dims(d["Q"], d["K"])
+    Y = torch.empty_like(d["X"])
+    Lk = torch.empty(dm.B, dtype=torch.int32, device=dev)
+    st = torch.cuda.current_stream(dev)
+    for q in (16, 64):
+        ws = tsa.workspace(dm, q, layer=True, device=dev)
+        for tau in (0.002, 0.005, 0.01, 0.02):
+            run = lambda: tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=q, tau=tau,
+                                        Lkeep=Lk, ws=ws)
+            for _ in range(2):
+                run()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            torch.cuda.synchronize()
+            ev[0].record(st)
+            for _ in range(3):
+                run()
+            ev[1].record(st)
+            torch.cuda.synchronize()
+            if tsa.tsa_get_device_status(ws) != 0:
+                raise RuntimeError("device error in the sweep")
+            ms = ev[0].elapsed_time(ev[1]) / 3
+            lks = [int(v) for v in Lk.cpu()]
+            fl = sum(2.0 * dm.H * dm.d * k * (k + 1) for k in lks)
+            print(json.dumps({
+                "metric": "token-sparse attn layer ms, tau x q sweep", "value": ms, "unit": "ms",
+                "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": _workload_desc(WORKLOADS[name], dm.L), "tau": tau,
+                           "q": q, "B": dm.B},
+                "Lkeep": lks, "kept_fraction": [k / dm.L for k in lks],
+                "layer_tflops": fl / (ms * 1e-3) / 1e12}), flush=True)
+        del ws
 
 
 def main():
@@ -414,6 +593,10 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-pages-sparsity", action="store_true")
+    ap.add_argument("--stack", action="store_true",
+                    help="32-layer stack with the sparse set chosen by the drift pass")
+    ap.add_argument("--sweep", action="store_true", help="tau x q sweep, B = 2, L = 64K")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
@@ -424,6 +607,12 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.stack:
+        run_stack(args, args.L or 4096)
+        return
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":  # rank 0 alone times the oracle; other ranks exit
         run_reference(args, w, L, rank, world)
         return
