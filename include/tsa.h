@@ -166,6 +166,21 @@ TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K,
                      int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
                      void *const *stage_events);
 
+/* Compress, attention and decompress in one pass ([notes] 关键设计 1: the compressed
+ * Q̂K̂V̂ are the rows S_h of Q, K, V; Decompress writes Ô back into those rows): the same
+ * result as tsa_gather_qkv + tsa_attn + tsa_scatter_residual, bit for bit, without the
+ * compressed copies.  The attention kernel reads the rows idx[b,h,0:Lkeep[b]] of Q
+ * [B,L,H,d] and of K, V [B,L,Hkv,d] (KV head h / (H / Hkv)) directly, and its epilogue
+ * writes Y[b,t,h*d:(h+1)*d] = X + bf16(Ô) (fp32 add, one rounding) for every kept token
+ * t; the other segments of Y are copied from X (nothing to do when Y == X).  idx as
+ * tsa_select writes it (kept tokens ascending, then the rest); an index outside [0, L)
+ * is reported in the workspace's error word.  bf16 only (TSA_ERR_UNSUPPORTED for fp32).
+ * ws supplies the error word (>= 256 bytes). */
+TSA_API tsa_status tsa_attn_gather(const tsa_dims *dims, const void *Q, const void *K,
+                                   const void *V, const int32_t *idx, const int32_t *Lkeep,
+                                   float scale, const void *X, void *Y, void *ws,
+                                   size_t ws_bytes, void *stream);
+
 /* ---- Budget and score variants ([notes] 消融实验 and 关键设计 2) ------------------- */
 
 typedef enum { TSA_POOL_NONE = 0, TSA_POOL_MAX = 1, TSA_POOL_MEAN = 2 } tsa_pool_kind;
@@ -199,8 +214,10 @@ typedef struct {
     int32_t budget;     /* tsa_budget_kind                      */
     double tau;         /* coverage threshold, [0, 1)           */
     double sparsity;    /* fixed fraction pruned, [0, 1]        */
-    int32_t pool;       /* tsa_pool_kind                        */
-    int32_t pool_width; /* odd, 1..255 (ignored for POOL_NONE)  */
+    int32_t pool;          /* tsa_pool_kind                        */
+    int32_t pool_width;    /* odd, 1..255 (ignored for POOL_NONE)  */
+    int32_t direct_gather; /* 1: tsa_attn_gather instead of gather, attention, scatter
+                              (bf16 only; same Y bit for bit)      */
 } tsa_layer_opts;
 
 /* tsa_layer with the budget and score variants of tsa_layer_opts (opts NULL: coverage

@@ -162,3 +162,54 @@ def test_drift_llama_width_32_layers():
         h.append(h[-1] * 0.9 + (0.05 + 0.01 * (l % 7)) * torch.randn(T, D, generator=g))
     R, mask = _drift_check(torch.stack(h).to(torch.bfloat16).contiguous())
     assert mask.sum() == 16
+
+
+# ---------------------------------------------------------------- direct-gather attention
+def _staged(d, dm, Lk, idx):
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk)
+    Oh = tsa.tsa_attn(dm, Qh, Kh, Vh, Lk)
+    return tsa.tsa_scatter_residual(dm, Oh, idx, Lk, d["X"])
+
+
+@pytest.mark.parametrize("B,L,H,Hkv", [(1, 4096, 32, 8), (2, 1000, 8, 2), (2, 5000, 8, 8)])
+def test_attn_gather_equals_staged_path_bitwise(B, L, H, Hkv):
+    x = make_inputs(B, L, H, Hkv, 128, torch.bfloat16, seed=L + H)
+    d = {k: v.cuda() for k, v in x.items()}
+    dm = tsa.dims(d["Q"], d["K"])
+    s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16)
+    for keep in (None, [0] * B, [1] * B, [L] * B, [L // 3 + 7 * b for b in range(B)]):
+        Lk = (tsa.tsa_budget(dm, s_l, 0.02) if keep is None
+              else torch.tensor(keep, dtype=torch.int32, device="cuda"))
+        idx = tsa.tsa_select(dm, s_h, Lk)
+        want = _staged(d, dm, Lk, idx)
+        ws = tsa.workspace(dm, 1)
+        got = tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, d["X"], ws=ws)
+        Yi = d["X"].clone()
+        tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, Yi, Yi, ws=ws)
+        assert tsa.tsa_get_device_status(ws) == 0
+        assert torch.equal(got, want), keep
+        assert torch.equal(Yi, want), keep
+        if keep is not None and keep[0] == 0:
+            assert torch.equal(got, d["X"])
+
+
+def test_layer_direct_gather_equals_staged_layer():
+    x = make_inputs(2, 3000, 32, 8, 128, torch.bfloat16, seed=77)
+    d = {k: v.cuda() for k, v in x.items()}
+    Y1 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, tau=0.01)
+    Y2 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, tau=0.01, direct=True)
+    Y3 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, sparsity=0.5, direct=True)
+    Y4 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, sparsity=0.5)
+    assert torch.equal(Y1, Y2) and torch.equal(Y3, Y4)
+
+
+def test_attn_gather_reports_a_bad_index():
+    x = make_inputs(1, 512, 4, 4, 128, torch.bfloat16, seed=5)
+    d = {k: v.cuda() for k, v in x.items()}
+    dm = tsa.dims(d["Q"], d["K"])
+    idx = torch.arange(512, dtype=torch.int32, device="cuda").repeat(1, 4, 1).contiguous()
+    idx[0, 2, 10] = 512                      # out of range: skipped and reported
+    Lk = torch.tensor([512], dtype=torch.int32, device="cuda")
+    ws = tsa.workspace(dm, 1)
+    tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, d["X"], ws=ws)
+    assert tsa.tsa_get_device_status(ws) == 1            # TSA_ERR_INVALID_ARG

@@ -19,6 +19,11 @@ cudaError_t launch_score_tc(const tsa_dims &, const void *, const void *, int, f
                             const WsLayout &, char *, cudaStream_t, uint32_t);
 cudaError_t launch_fill_lkeep(int, int32_t, int32_t *, cudaStream_t);
 size_t drift_workspace_bytes(int, long long);
+cudaError_t launch_attn_gather(const tsa_dims &, const void *, const void *, const void *,
+                               const int32_t *, const int32_t *, float, const void *, void *,
+                               Control *, cudaStream_t, uint32_t);
+cudaError_t launch_copy_rest(const tsa_dims &, const int32_t *, const int32_t *, const void *,
+                             void *, cudaStream_t);
 cudaError_t launch_drift(int, long long, int, int, const void *, double, double, double *,
                          int32_t *, char *, cudaStream_t);
 cudaError_t launch_pool(const tsa_dims &, const float *, int, int, float *, cudaStream_t);
@@ -330,6 +335,36 @@ tsa_status tsa_pool_scores(const tsa_dims *dims, const float *s_h, int32_t kind,
                        "tsa_pool_scores (normalise)");
 }
 
+// Fused compress + attention + decompress: rows through idx, Y = X + Ô in the kept rows,
+// Y = X in the others (copied when Y != X).
+static tsa_status do_attn_gather(const tsa_dims &dm, const void *Q, const void *K,
+                                 const void *V, const int32_t *idx, const int32_t *Lkeep,
+                                 float scale, const void *X, void *Y, char *ws, cudaStream_t st) {
+    if (X != Y)
+        TSA_TRY(cuda_status(launch_copy_rest(dm, idx, Lkeep, X, Y, st), "tsa_attn_gather (rest)"));
+    return cuda_status(launch_attn_gather(dm, Q, K, V, idx, Lkeep, scale, X, Y, (Control *)ws, st,
+                                          g_wait_limit_us),
+                       "tsa_attn_gather");
+}
+
+tsa_status tsa_attn_gather(const tsa_dims *dims, const void *Q, const void *K, const void *V,
+                           const int32_t *idx, const int32_t *Lkeep, float scale, const void *X,
+                           void *Y, void *ws, size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    if (dims->dtype != TSA_BF16)
+        return fail(TSA_ERR_UNSUPPORTED, "tsa_attn_gather runs the bf16 tensor-core path only");
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_ptr(Q, "Q"));
+    TSA_TRY(check_ptr(K, "K"));
+    TSA_TRY(check_ptr(V, "V"));
+    TSA_TRY(check_ptr(idx, "idx"));
+    TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    TSA_TRY(check_ptr(X, "X"));
+    TSA_TRY(check_ptr(Y, "Y"));
+    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
+    return do_attn_gather(*dims, Q, K, V, idx, Lkeep, scale, X, Y, (char *)ws, (cudaStream_t)stream);
+}
+
 static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K, const void *V,
                              const void *X, void *Y, int32_t is_sparse, int32_t q,
                              const tsa_layer_opts &o, float scale, float *s_h_out,
@@ -346,6 +381,8 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
         return fail(TSA_ERR_INVALID_ARG, "unknown budget kind");
     }
     if (o.pool != TSA_POOL_NONE) TSA_TRY(check_pool(o.pool, o.pool_width));
+    if (o.direct_gather && dims->dtype != TSA_BF16)
+        return fail(TSA_ERR_UNSUPPORTED, "direct gather runs the bf16 tensor-core path only");
     TSA_TRY(check_ptr(Q, "Q"));
     TSA_TRY(check_ptr(K, "K"));
     TSA_TRY(check_ptr(V, "V"));
@@ -395,6 +432,12 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
     TSA_TRY(rec(2));
     TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, w, st), "tsa_layer select"));
     TSA_TRY(rec(3));
+    if (o.direct_gather) {  // no compressed copies: one fused attention pass
+        TSA_TRY(rec(4));
+        TSA_TRY(do_attn_gather(dm, Q, K, V, idx, Lk, scale, X, Y, w, st));
+        TSA_TRY(rec(5));
+        return rec(6);
+    }
     TSA_TRY(cuda_status(launch_gather(dm, Q, K, V, idx, Lk, Qh, Kh, Vh, (Control *)w, st),
                         "tsa_layer gather"));
     TSA_TRY(rec(4));
@@ -409,7 +452,7 @@ tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const v
                      float scale, float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
                      int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
                      void *const *stage_events) {
-    tsa_layer_opts o{TSA_BUDGET_COVERAGE, tau, 0.0, TSA_POOL_NONE, 1};
+    tsa_layer_opts o{TSA_BUDGET_COVERAGE, tau, 0.0, TSA_POOL_NONE, 1, 0};
     return layer_impl(dims, Q, K, V, X, Y, is_sparse, q, o, scale, s_h_out, s_l_out, Lkeep_out,
                       idx_out, ws, ws_bytes, stream, stage_events);
 }
@@ -420,7 +463,7 @@ tsa_status tsa_layer_ex(const tsa_dims *dims, const void *Q, const void *K, cons
                         float *s_l_out, int32_t *Lkeep_out, int32_t *idx_out, void *ws,
                         size_t ws_bytes, void *stream, void *const *stage_events) {
     const tsa_layer_opts o = opts ? *opts
-                                  : tsa_layer_opts{TSA_BUDGET_COVERAGE, 0.005, 0.0, TSA_POOL_NONE, 1};
+                                  : tsa_layer_opts{TSA_BUDGET_COVERAGE, 0.005, 0.0, TSA_POOL_NONE, 1, 0};
     return layer_impl(dims, Q, K, V, X, Y, is_sparse, q, o, scale, s_h_out, s_l_out, Lkeep_out,
                       idx_out, ws, ws_bytes, stream, stage_events);
 }

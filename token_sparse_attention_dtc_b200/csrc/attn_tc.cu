@@ -26,6 +26,7 @@
 // Every wait is bounded in time; a wait that runs out records TSA_ERR_DEVICE_TIMEOUT,
 // the CTA drains its in-flight copies and MMAs, frees TMEM and exits.
 #include <math.h>
+#include <string.h>
 
 #include <algorithm>
 
@@ -47,10 +48,112 @@ template <int D> struct AttnSmem {
     uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], o_final[2], drain;
     uint64_t stall;  // test hook: initialised, never completed
+    int32_t gidx[2][kBM];  // direct-gather mode: token indices of the tiles being copied
     uint32_t tmem_base;
     int abort;
     int never;  // stays 0: drain waits ignore the abort flag
 };
+
+// Direct-gather mode: rows are read through the index lists from the original tensors,
+// and the epilogue writes Y = X + Ô into the kept rows (no compressed copies).
+struct GatherArgs {
+    const __nv_bfloat16 *Q, *K, *V;  // [B, L, H, d], [B, L, Hkv, d]
+    const int32_t *idx;              // [B, H, L]: kept tokens ascending, then the rest
+    const __nv_bfloat16 *X;          // [B, L, H*d]
+    __nv_bfloat16 *Y;                // [B, L, H*d], may be X
+};
+
+// Producer of the direct-gather mode (all 32 lanes of warp 0).  A 128-row tile of
+// positions p0..p0+127 is copied with 16-byte cp.async into the 128-byte-swizzle layout
+// the MMA descriptors read (16-byte chunk k of row r at r*128 + ((k ^ (r & 7)) * 16) in
+// each 64-column block), row p taken from token idx[p] (p clamped to L - 1; rows past L'
+// are masked or never stored).  One commit group per tile; once the group before the
+// newest has landed, each lane fences (generic -> async proxy) and arrives on its full
+// barrier (32 arrivals).
+template <int D>
+__device__ __forceinline__ bool gather_producer(AttnSmem<D> &sm, const GatherArgs &ga, int b,
+                                                int h, int kvh, int L, int H, int Hkv, int i0,
+                                                bool hasB, int nkv, int lane, Control *ctl,
+                                                uint64_t limit_ns, volatile int *abort) {
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    const int32_t *S = ga.idx + ((size_t)b * H + h) * L;
+    bool bad = false;
+    // Token indices of rows p0 + 4*lane .. p0 + 4*lane + 3 (clamped to L - 1), loaded in
+    // one round trip; staged in shared memory so the copy loop has no global dependence.
+    auto load_idx = [&](int p0, int (&v)[4]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = __ldg(S + min(p0 + 4 * lane + e, L - 1));
+    };
+    auto stage_idx = [&](int slot, const int (&v)[4]) {
+        __syncwarp();  // the previous copy loop has read this slot
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            int t = v[e];
+            if ((unsigned)t >= (unsigned)L) {
+                bad = true;
+                t = 0;
+            }
+            sm.gidx[slot][4 * lane + e] = t;
+        }
+        __syncwarp();
+    };
+    auto tile = [&](uint8_t *dst, const __nv_bfloat16 *src, int heads, int head, int slot) {
+        const uint32_t d0 = smem_u32(dst);
+        const int c = lane % CPR;
+        const uint32_t coff = (uint32_t)(c / 8) * (kBM * 128);
+        const __nv_bfloat16 *base = src + (size_t)head * D + c * 8;
+#pragma unroll 8
+        for (int r = lane / CPR; r < kBM; r += 32 / CPR) {
+            const int t = sm.gidx[slot][r];
+            cp_async16(d0 + coff + r * 128 + (((c % 8) ^ (r & 7)) << 4),
+                       base + ((size_t)b * L + t) * heads * D);
+        }
+    };
+    uint64_t *pending = nullptr;
+    auto publish_previous = [&]() {
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        if (pending) mbar_arrive(pending);
+    };
+    int va[4], vb[4];
+    load_idx(i0, va);
+    if (hasB) load_idx(i0 + kBM, vb);
+    stage_idx(0, va);
+    tile(sm.q[0], ga.Q, H, h, 0);
+    if (hasB) {
+        stage_idx(1, vb);
+        tile(sm.q[1], ga.Q, H, h, 1);
+    }
+    cp_async_commit();
+    pending = &sm.q_full;
+    int nxt[4];
+    if (nkv > 0) load_idx(0, nxt);
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+        const int s = j % kStages, slot = j & 1;
+        const uint32_t ph = ((j / kStages) & 1) ^ 1;
+        stage_idx(slot, nxt);
+        if (j + 1 < nkv) load_idx((j + 1) * kBN, nxt);  // in flight during this step's copies
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.k_empty[s], ph, limit_ns, abort));
+        if (!ok) break;
+        tile(sm.k[s], ga.K, Hkv, kvh, slot);
+        cp_async_commit();
+        publish_previous();
+        pending = &sm.k_full[s];
+        ok = __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[s], ph, limit_ns, abort));
+        if (!ok) break;
+        tile(sm.v[s], ga.V, Hkv, kvh, slot);
+        cp_async_commit();
+        publish_previous();
+        pending = &sm.v_full[s];
+    }
+    // Drain: every copy of this lane lands before the CTA can exit; publish the last tile.
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (ok) mbar_arrive(pending);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(ctl, TSA_ERR_INVALID_ARG, 31);
+    return ok;
+}
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
@@ -151,12 +254,12 @@ __device__ __forceinline__ bool softmax_tile(AttnSmem<D> &sm, int X, int n, uint
     return true;
 }
 
-template <int D>
+template <int D, bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ Lkeep, int dense,
-          int L, int H, int Hkv, float sl2, __nv_bfloat16 *__restrict__ O, Control *ctl,
-          uint64_t limit_ns, int stall) {
+          int L, int H, int Hkv, float sl2, __nv_bfloat16 *__restrict__ O, GatherArgs ga,
+          Control *ctl, uint64_t limit_ns, int stall) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem<D> &sm = *reinterpret_cast<AttnSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -172,15 +275,16 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const bool hasB = i0 + kBM < Lk;
     const int nA = 2 * pair + 1, nB = hasB ? 2 * pair + 2 : 0;
     const int nkv = hasB ? nB : nA;
-    const int kvh = dense ? h / (H / Hkv) : h;
+    const int kvh = (dense || kGather) ? h / (H / Hkv) : h;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(&sm.q_full, 1);
+        const uint32_t nfill = kGather ? 32 : 1;  // cp.async lanes, or one TMA thread
+        mbar_init(&sm.q_full, nfill);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.k_full[s], nfill);
             mbar_init(&sm.k_empty[s], 1);
-            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.v_full[s], nfill);
             mbar_init(&sm.v_empty[s], 1);
         }
         for (int x = 0; x < 2; ++x) {
@@ -204,7 +308,10 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort = &sm.abort;
     bool ok = true;
-    if (warp == 0) {
+    if (warp == 0 && kGather) {
+        ok = gather_producer<D>(sm, ga, b, h, kvh, L, H, Hkv, i0, hasB, nkv, lane, ctl, limit_ns,
+                                abort);
+    } else if (warp == 0) {
         if (lane == 0) {
             int issued = 0;  // K/V tiles issued (negative: K of tile -issued-1 only)
             mbar_expect_tx(&sm.q_full, 2 * TILE);
@@ -319,6 +426,38 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const float inv = 1.0f / l;
                 __nv_bfloat16 *orow = dense ? O + (((size_t)b * L + i) * H + h) * D
                                             : O + ((size_t)bh * L + i) * D;
+                if (kGather) {  // Y[t] = X[t] + bf16(O / l) for token t = idx[i]
+                    const int t = i < Lk ? __ldg(ga.idx + (size_t)bh * L + i) : -1;
+                    const bool st = (unsigned)t < (unsigned)L;
+                    const size_t seg = st ? (((size_t)b * L + t) * H + h) * D : 0;
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + lo + c * 32, o);
+                        tmem_ld_wait();
+                        if (st) {
+                            const uint4 *xs = reinterpret_cast<const uint4 *>(ga.X + seg + c * 32);
+                            uint4 *ys = reinterpret_cast<uint4 *>(ga.Y + seg + c * 32);
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                const uint4 xv = xs[q4];
+                                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                                uint32_t yw[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const uint32_t ob = pack_bf16(
+                                        __uint_as_float(o[q4 * 8 + 2 * e]) * inv,
+                                        __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv);
+                                    yw[e] = pack_bf16(
+                                        __uint_as_float(xw[e] << 16) + __uint_as_float(ob << 16),
+                                        __uint_as_float(xw[e] & 0xffff0000u) +
+                                            __uint_as_float(ob & 0xffff0000u));
+                                }
+                                ys[q4] = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+                            }
+                        }
+                    }
+                } else {
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
@@ -341,6 +480,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                         }
                     }
                 }
+                }
             } else {
                 ok = false;
             }
@@ -360,15 +500,20 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 
 }  // namespace
 
-template <int D>
+template <int D, bool kGather>
 static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                                 const int32_t *Lkeep, int dense, float scale, void *O,
-                                Control *ctl, cudaStream_t st, uint32_t limit_us) {
+                                const GatherArgs &ga, Control *ctl, cudaStream_t st,
+                                uint32_t limit_us) {
     CUtensorMap tq, tk, tv;
+    memset(&tq, 0, sizeof tq);  // the direct-gather mode reads no tensor map
+    memset(&tk, 0, sizeof tk);
+    memset(&tv, 0, sizeof tv);
     const uint64_t B = dm.B, L = dm.L, H = dm.H, Hkv = dm.Hkv;
     const uint32_t box[4] = {64, (uint32_t)kBM, 1, 1};
-    bool okm;
-    if (dense) {
+    bool okm = true;
+    if (kGather) {
+    } else if (dense) {
         const uint64_t dq[4] = {(uint64_t)D, L, H, B}, dk[4] = {(uint64_t)D, L, Hkv, B};
         const uint64_t sq[3] = {H * D * 2, (uint64_t)D * 2, L * H * D * 2};
         const uint64_t sk[3] = {Hkv * D * 2, (uint64_t)D * 2, L * Hkv * D * 2};
@@ -383,13 +528,13 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
     if (!okm) return cudaErrorInvalidValue;
     // At least 116 KB so that one CTA holds an SM (and all 512 TMEM columns) at a time.
     const size_t smem = std::max<size_t>(sizeof(AttnSmem<D>) + 1024, 116 * 1024);
-    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D, kGather>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long nblocks = (long)ceil_div(dm.L, 2 * kBM) * dm.B * dm.H;
-    k_attn_tc<D><<<(unsigned)nblocks, kThreads, smem, st>>>(
+    k_attn_tc<D, kGather><<<(unsigned)nblocks, kThreads, smem, st>>>(
         tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
-        (__nv_bfloat16 *)O, ctl, (uint64_t)limit_us * 1000ull, test_stall());
+        (__nv_bfloat16 *)O, ga, ctl, (uint64_t)limit_us * 1000ull, test_stall());
     note_launches(1);
     return cudaGetLastError();
 }
@@ -397,8 +542,30 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
 cudaError_t launch_attn_tc(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                            const int32_t *Lkeep, int dense, float scale, void *O, Control *ctl,
                            cudaStream_t st, uint32_t limit_us) {
-    return dm.d == 64 ? attn_tc_impl<64>(dm, Q, K, V, Lkeep, dense, scale, O, ctl, st, limit_us)
-                      : attn_tc_impl<128>(dm, Q, K, V, Lkeep, dense, scale, O, ctl, st, limit_us);
+    const GatherArgs none{};
+    return dm.d == 64
+               ? attn_tc_impl<64, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, ctl, st, limit_us)
+               : attn_tc_impl<128, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, ctl, st,
+                                          limit_us);
+}
+
+// Compressed attention reading Q, K, V rows through idx, with Y = X + Ô written into the
+// kept rows (the unselected rows of Y are the caller's: equal to X in place).
+cudaError_t launch_attn_gather(const tsa_dims &dm, const void *Q, const void *K, const void *V,
+                               const int32_t *idx, const int32_t *Lkeep, float scale,
+                               const void *X, void *Y, Control *ctl, cudaStream_t st,
+                               uint32_t limit_us) {
+    GatherArgs ga;
+    ga.Q = (const __nv_bfloat16 *)Q;
+    ga.K = (const __nv_bfloat16 *)K;
+    ga.V = (const __nv_bfloat16 *)V;
+    ga.idx = idx;
+    ga.X = (const __nv_bfloat16 *)X;
+    ga.Y = (__nv_bfloat16 *)Y;
+    return dm.d == 64
+               ? attn_tc_impl<64, true>(dm, Q, K, V, Lkeep, 0, scale, nullptr, ga, ctl, st, limit_us)
+               : attn_tc_impl<128, true>(dm, Q, K, V, Lkeep, 0, scale, nullptr, ga, ctl, st,
+                                         limit_us);
 }
 
 }  // namespace tsa

@@ -120,6 +120,25 @@ k_scatter_residual(const uint4 *__restrict__ Oh, const int32_t *__restrict__ idx
     }
 }
 
+// The unselected segments of an out-of-place layer whose kept segments the attention
+// epilogue writes itself: Y[seg] = X[seg] for idx[Lk:L].  grid (B*H, ceil(L / kGatherRows)).
+template <int VPR>
+__global__ void __launch_bounds__(kMoveThreads)
+k_copy_rest(const int32_t *__restrict__ idx, const int32_t *__restrict__ Lkeep, const uint4 *X,
+            uint4 *Y, int L, int H) {
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int Lk = Lkeep[b];
+    const int i0 = max(blockIdx.y * kGatherRows, Lk), i1 = min(L, (blockIdx.y + 1) * kGatherRows);
+    const int32_t *S = idx + (size_t)bh * L;
+    for (int e = threadIdx.x; e < (i1 - i0) * VPR; e += kMoveThreads) {
+        const int i = i0 + e / VPR, v = e % VPR;
+        const int t = S[i];
+        if ((unsigned)t >= (unsigned)L) continue;  // a bad list is reported by the attention
+        const size_t seg = (((size_t)b * L + t) * H + h) * VPR + v;
+        Y[seg] = X[seg];
+    }
+}
+
 // Dense residual: Y = X + O elementwise over [B, L, H*d].
 template <typename T>
 __global__ void __launch_bounds__(kMoveThreads)
@@ -187,6 +206,20 @@ cudaError_t launch_scatter(const tsa_dims &dm, const void *Oh, const int32_t *id
                            const int32_t *Lkeep, const void *X, void *Y, cudaStream_t st) {
     return dm.dtype == TSA_F32 ? scatter_impl<float>(dm, Oh, idx, Lkeep, X, Y, st)
                                : scatter_impl<__nv_bfloat16>(dm, Oh, idx, Lkeep, X, Y, st);
+}
+
+cudaError_t launch_copy_rest(const tsa_dims &dm, const int32_t *idx, const int32_t *Lkeep,
+                             const void *X, void *Y, cudaStream_t st) {
+    const int vpr = dm.d * (dm.dtype == TSA_F32 ? 4 : 2) / 16;
+    dim3 grid(dm.B * dm.H, ceil_div(dm.L, kGatherRows));
+    switch (vpr) {
+        case 8: k_copy_rest<8><<<grid, kMoveThreads, 0, st>>>(idx, Lkeep, (const uint4 *)X, (uint4 *)Y, dm.L, dm.H); break;
+        case 16: k_copy_rest<16><<<grid, kMoveThreads, 0, st>>>(idx, Lkeep, (const uint4 *)X, (uint4 *)Y, dm.L, dm.H); break;
+        case 32: k_copy_rest<32><<<grid, kMoveThreads, 0, st>>>(idx, Lkeep, (const uint4 *)X, (uint4 *)Y, dm.L, dm.H); break;
+        default: return cudaErrorInvalidValue;
+    }
+    note_launches(1);
+    return cudaGetLastError();
 }
 
 }  // namespace tsa

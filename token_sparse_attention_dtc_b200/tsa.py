@@ -25,7 +25,7 @@ EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_b
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
            "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall",
            "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex",
-           "tsa_drift_workspace_size", "tsa_drift")
+           "tsa_drift_workspace_size", "tsa_drift", "tsa_attn_gather")
 POOL_NONE, POOL_MAX, POOL_MEAN = 0, 1, 2
 BUDGET_COVERAGE, BUDGET_FIXED = 0, 1
 
@@ -45,7 +45,7 @@ class LayerOpts(ctypes.Structure):
     """tsa_layer_opts of include/tsa.h."""
     _fields_ = [("budget", ctypes.c_int32), ("tau", ctypes.c_double),
                 ("sparsity", ctypes.c_double), ("pool", ctypes.c_int32),
-                ("pool_width", ctypes.c_int32)]
+                ("pool_width", ctypes.c_int32), ("direct_gather", ctypes.c_int32)]
 
 
 def lib():
@@ -76,6 +76,7 @@ def lib():
             "tsa_last_error": (ctypes.c_char_p, []),
             "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
             "tsa_budget_fixed": (I32, [DP, D, P, P]),
+            "tsa_attn_gather": (I32, [DP, P, P, P, P, P, F, P, P, P, SZ, P]),
             "tsa_drift_workspace_size": (SZ, [I32, ctypes.c_int64]),
             "tsa_drift": (I32, [I32, ctypes.c_int64, I32, I32, P, D, D, P, P, P, SZ, P]),
             "tsa_pool_scores": (I32, [DP, P, I32, I32, P, P, P, SZ, P]),
@@ -246,6 +247,21 @@ def tsa_drift(h, eps: float = 1e-6, delta: float = 0.5, ws=None, stream=None):
     return R, mask
 
 
+def tsa_attn_gather(Q, K, V, idx, Lkeep, X, Y=None, scale: float | None = None, ws=None,
+                    stream=None):
+    """Fused compress + attention + decompress: returns Y (= X + Decompress(Ô))."""
+    dm = dims(Q, K)
+    _need_cuda(Q, K, V, idx, Lkeep, X)
+    if Y is None:
+        Y = torch.empty_like(X)
+    if ws is None:
+        ws = workspace(dm, 1, device=Q.device)
+    _check(lib().tsa_attn_gather(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(idx), _p(Lkeep),
+                                 default_scale(dm.d) if scale is None else scale, _p(X), _p(Y),
+                                 _p(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
 def tsa_budget_fixed(dm: Dims, sparsity: float, Lkeep=None, device=None, stream=None):
     """Fixed-ratio budget: Lkeep[b] = L - floor(sparsity * L)."""
     if Lkeep is None:
@@ -273,10 +289,11 @@ def tsa_pool_scores(dm: Dims, s_h, kind: int, width: int, s_h_out=None, s_l_out=
 def tsa_layer(Q, K, V, X, Y=None, is_sparse: bool = True, q: int = 16, tau: float = 0.005,
               scale: float | None = None, s_h=None, s_l=None, Lkeep=None, idx=None, ws=None,
               stream=None, stage_events=None, sparsity: float | None = None,
-              pool: int = POOL_NONE, pool_width: int = 1):
+              pool: int = POOL_NONE, pool_width: int = 1, direct: bool = False):
     """One Token Sparse Attention layer: returns Y = X + Decompress(Ô) (or the dense layer).
     sparsity (fixed-ratio budget instead of tau) and pool / pool_width (pooled head
-    scores) select the variants of tsa_layer_ex."""
+    scores) and direct (fused compress + attention + decompress) select the variants of
+    tsa_layer_ex."""
     dm = dims(Q, K)
     _need_cuda(Q, K, V, X, Y, s_h, s_l, Lkeep, idx)
     if Y is None:
@@ -287,13 +304,14 @@ def tsa_layer(Q, K, V, X, Y=None, is_sparse: bool = True, q: int = 16, tau: floa
     if stage_events is not None:
         ev = (ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
     sc = default_scale(dm.d) if scale is None else scale
-    if sparsity is None and pool == POOL_NONE:
+    if sparsity is None and pool == POOL_NONE and not direct:
         _check(lib().tsa_layer(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y),
                                int(is_sparse), q, float(tau), sc, _p(s_h), _p(s_l), _p(Lkeep),
                                _p(idx), _p(ws), ws.numel(), _stream(stream), ev))
         return Y
     o = LayerOpts(BUDGET_COVERAGE if sparsity is None else BUDGET_FIXED, float(tau),
-                  0.0 if sparsity is None else float(sparsity), int(pool), int(pool_width))
+                  0.0 if sparsity is None else float(sparsity), int(pool), int(pool_width),
+                  int(bool(direct)))
     _check(lib().tsa_layer_ex(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y),
                               int(is_sparse), q, ctypes.byref(o), sc, _p(s_h), _p(s_l),
                               _p(Lkeep), _p(idx), _p(ws), ws.numel(), _stream(stream), ev))
