@@ -51,9 +51,13 @@ def _load():
         lib.orc_pool.argtypes = [I, I, I, P, I, I, P, P]
         lib.orc_drift.argtypes = [I, L, I, I, P, D, P]
         lib.orc_drift_mask.argtypes = [I, P, D, P]
+        lib.orc_block_logits.argtypes = [I, I, I, I, I, I, P, P, P, P, D, P]
+        lib.orc_block_select.argtypes = [I, I, I, P, P, ctypes.c_float, P]
+        lib.orc_attend_block_rows.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, D, P, L, P]
         for f in ("orc_score", "orc_budget", "orc_select", "orc_attend_rows",
                   "orc_decompress_residual", "orc_budget_fixed", "orc_pool", "orc_drift",
-                  "orc_drift_mask"):
+                  "orc_drift_mask", "orc_block_logits", "orc_block_select",
+                  "orc_attend_block_rows"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -172,6 +176,55 @@ def drift_mask(R, delta: float = 0.5):
     if rc:
         raise ValueError("orc_drift_mask rejected its arguments (%d)" % rc)
     return mask
+
+
+def block_logits(Q, K, idx, Lkeep, scale: float | None = None):
+    """Block logits z [B, H, ceil(L/256), ceil(L/128)] fp64 of the block-sparse pattern
+    (NaN where a pair or block does not exist)."""
+    q, k = _np(Q), _np(K)
+    B, L, H, d = q.shape
+    Hkv = k.shape[2]
+    ix = np.ascontiguousarray(_np(idx), dtype=np.int32)
+    lk = np.ascontiguousarray(_np(Lkeep), dtype=np.int32)
+    z = np.zeros((B, H, (L + 255) // 256, (L + 127) // 128), np.float64)
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    rc = _load().orc_block_logits(B, L, H, Hkv, d, _dtype_code(q), _ptr(q), _ptr(k), _ptr(ix),
+                                  _ptr(lk), float(sc), _ptr(z))
+    if rc:
+        raise ValueError("orc_block_logits rejected its arguments (%d)" % rc)
+    return z
+
+
+def block_select(z, Lkeep, theta: float):
+    """Kept blocks uint8 [B, H, NP, NB] from fp32 block logits z (fp32 threshold)."""
+    zz = np.ascontiguousarray(_np(z), dtype=np.float32)
+    B, H, NP, NB = zz.shape
+    lk = np.ascontiguousarray(_np(Lkeep), dtype=np.int32)
+    keep = np.zeros((B, H, NP, NB), np.uint8)
+    L = NB * 128
+    rc = _load().orc_block_select(B, H, L, _ptr(lk), _ptr(zz), ctypes.c_float(theta), _ptr(keep))
+    if rc:
+        raise ValueError("orc_block_select rejected its arguments (%d)" % rc)
+    return keep
+
+
+def attend_block_rows(Q, K, V, idx, Lkeep, keep, rows, scale: float | None = None):
+    """Block-sparse attention rows Ô[b, h, i] for rows [(b, h, i), ...]; fp64 [n, d]."""
+    q, k, v = _np(Q), _np(K), _np(V)
+    B, L, H, d = q.shape
+    ix = np.ascontiguousarray(_np(idx), dtype=np.int32)
+    lk = np.ascontiguousarray(_np(Lkeep), dtype=np.int32)
+    kp = np.ascontiguousarray(keep, dtype=np.uint8)
+    assert kp.shape[2:] == ((L + 255) // 256, (L + 127) // 128)
+    r = np.ascontiguousarray(np.asarray(rows, np.int32).reshape(-1, 3))
+    out = np.zeros((len(r), d), np.float64)
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    rc = _load().orc_attend_block_rows(B, L, H, k.shape[2], d, _dtype_code(q), _ptr(q), _ptr(k),
+                                       _ptr(v), _ptr(ix), _ptr(lk), _ptr(kp), float(sc), _ptr(r),
+                                       len(r), _ptr(out))
+    if rc:
+        raise ValueError("orc_attend_block_rows rejected its arguments (%d)" % rc)
+    return out
 
 
 def select(s_h, Lkeep):

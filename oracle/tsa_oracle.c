@@ -444,3 +444,119 @@ int orc_drift_mask(int N, const double *R, double delta, int32_t *mask) {
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Block-sparse pattern inside the compressed space: [notes] 关键发现 (token  */
+/* sparsity stacked on block-level sparsity is the most valuable pairing)    */
+/* and [blog] §3.2 与现有方案的兼容性 ("token selection first, then block-    */
+/* sparse computation").  The block choice is this project's own definition: */
+/* the pages give none.  In head h's compressed                              */
+/* order (position i is token S_h[i]):                                       */
+/*   query pair p = positions [256p, 256p + 256), key block j = positions    */
+/*   [128j, 128j + 128);                                                     */
+/*   z[p][j] = scale * < mean of the pair's Q rows, mean of block j's K rows > */
+/*   for the blocks j < 2p before the pair's own (diagonal) blocks;         */
+/*   kept: j = 0, the diagonal blocks 2p and 2p + 1, and every j < 2p with   */
+/*   z[p][j] >= max_j z[p][j] - theta, the threshold taken in fp32 on fp32   */
+/*   logits (the precision the GPU decides in);                              */
+/*   attention: row i attends to the keys i' <= i whose block is kept for    */
+/*   the pair of i.                                                          */
+/* z has shape [B, H, NP, NB] with NP = ceil(L / 256), NB = ceil(L / 128);   */
+/* entries that do not exist are NaN.                                        */
+/* ------------------------------------------------------------------------ */
+int orc_block_logits(int B, int L, int H, int Hkv, int d, int dtype, const void *Q,
+                     const void *K, const int32_t *idx, const int32_t *Lkeep, double scale,
+                     double *z) {
+    if (B < 1 || L < 1 || H < 1 || Hkv < 1 || H % Hkv || d < 1) return 1;
+    const int NP = (L + 255) / 256, NB = (L + 127) / 128, G = H / Hkv;
+    double *qb = (double *)malloc(sizeof(double) * (size_t)d);
+    double *kb = (double *)malloc(sizeof(double) * (size_t)d);
+    for (size_t e = 0; e < (size_t)B * H * NP * NB; ++e) z[e] = NAN;
+    for (int b = 0; b < B; ++b) {
+        const int Lk = Lkeep[b];
+        for (int h = 0; h < H; ++h) {
+            const int32_t *S = idx + ((size_t)b * H + h) * L;
+            for (int p = 0; 256 * p < Lk; ++p) {
+                const int i1 = 256 * p + 256 < Lk ? 256 * p + 256 : Lk;
+                for (int c = 0; c < d; ++c) qb[c] = 0.0;
+                for (int i = 256 * p; i < i1; ++i)
+                    for (int c = 0; c < d; ++c)
+                        qb[c] += elem(Q, dtype, (((size_t)b * L + S[i]) * H + h) * d + c);
+                for (int c = 0; c < d; ++c) qb[c] /= (double)(i1 - 256 * p);
+                for (int j = 0; j < 2 * p; ++j) {
+                    for (int c = 0; c < d; ++c) kb[c] = 0.0;
+                    for (int i = 128 * j; i < 128 * j + 128; ++i)
+                        for (int c = 0; c < d; ++c)
+                            kb[c] += elem(K, dtype, (((size_t)b * L + S[i]) * Hkv + h / G) * d + c);
+                    double acc = 0.0;
+                    for (int c = 0; c < d; ++c) acc += qb[c] * (kb[c] / 128.0);
+                    z[(((size_t)b * H + h) * NP + p) * NB + j] = scale * acc;
+                }
+            }
+        }
+    }
+    free(qb);
+    free(kb);
+    return 0;
+}
+
+int orc_block_select(int B, int H, int L, const int32_t *Lkeep, const float *z, float theta,
+                     uint8_t *keep) {
+    if (B < 1 || H < 1 || L < 1 || !(theta >= 0.0f)) return 1;
+    const int NP = (L + 255) / 256, NB = (L + 127) / 128;
+    memset(keep, 0, (size_t)B * H * NP * NB);
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int p = 0; 256 * p < Lkeep[b]; ++p) {
+                const float *zr = z + (((size_t)b * H + h) * NP + p) * NB;
+                uint8_t *kr = keep + (((size_t)b * H + h) * NP + p) * NB;
+                kr[0] = 1;
+                kr[2 * p] = 1;
+                if (256 * p + 128 < Lkeep[b]) kr[2 * p + 1] = 1;
+                if (p == 0) continue;
+                float m = zr[0];
+                for (int j = 1; j < 2 * p; ++j) if (zr[j] > m) m = zr[j];
+                const float thr = m - theta; /* one fp32 subtraction */
+                for (int j = 1; j < 2 * p; ++j) if (zr[j] >= thr) kr[j] = 1;
+            }
+    return 0;
+}
+
+int orc_attend_block_rows(int B, int L, int H, int Hkv, int d, int dtype, const void *Q,
+                          const void *K, const void *V, const int32_t *idx,
+                          const int32_t *Lkeep, const uint8_t *keep, double scale,
+                          const int32_t *rows, long nrows, double *out) {
+    if (B < 1 || L < 1 || H < 1 || Hkv < 1 || H % Hkv || d < 1) return 1;
+    const int NP = (L + 255) / 256, NB = (L + 127) / 128, G = H / Hkv;
+    double *z = (double *)malloc(sizeof(double) * (size_t)L);
+    for (long r = 0; r < nrows; ++r) {
+        const int b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+        double *o = out + (size_t)r * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        if (i < 0 || i >= Lkeep[b]) continue;
+        const int32_t *S = idx + ((size_t)b * H + h) * L;
+        const uint8_t *kr = keep + (((size_t)b * H + h) * NP + i / 256) * NB;
+        const size_t qoff = (((size_t)b * L + S[i]) * H + h) * d;
+        double zmax = -INFINITY;
+        for (int jj = 0; jj <= i; ++jj) {
+            z[jj] = -INFINITY;
+            if (!kr[jj / 128]) continue;
+            const size_t koff = (((size_t)b * L + S[jj]) * Hkv + h / G) * d;
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += elem(Q, dtype, qoff + c) * elem(K, dtype, koff + c);
+            z[jj] = scale * acc;
+            if (z[jj] > zmax) zmax = z[jj];
+        }
+        double den = 0.0;
+        for (int jj = 0; jj <= i; ++jj) if (z[jj] != -INFINITY) den += exp(z[jj] - zmax);
+        for (int jj = 0; jj <= i; ++jj) {
+            if (z[jj] == -INFINITY) continue;
+            const double w = exp(z[jj] - zmax) / den;
+            const size_t voff = (((size_t)b * L + S[jj]) * Hkv + h / G) * d;
+            for (int c = 0; c < d; ++c) o[c] += w * elem(V, dtype, voff + c);
+        }
+    }
+    free(z);
+    return 0;
+}

@@ -442,3 +442,82 @@ def test_drift_rejects_bad_arguments():
         oracle.drift(np.zeros((1, 3, 4), np.float32))         # needs two states
     with pytest.raises(ValueError):
         oracle.drift_mask(np.zeros(3), 1.5)
+
+
+# ---------------------------------------------------------------- block-sparse pattern
+def _block_case(L=700, H=2, Hkv=1, d=16, seed=0, keep=None):
+    x = make_inputs(1, L, H, Hkv, d, torch.float32, seed=seed)
+    lk = np.array([L if keep is None else keep], np.int32)
+    rng = np.random.default_rng(seed)
+    idx = np.stack([np.concatenate([np.sort(p[:lk[0]]), np.sort(p[lk[0]:])])
+                    for p in (rng.permutation(L) for _ in range(H))])[None].astype(np.int32)
+    return x, idx, lk
+
+
+def test_block_logits_brute_force():
+    x, idx, lk = _block_case(L=600, keep=530)
+    z = oracle.block_logits(x["Q"], x["K"], idx, lk, scale=0.25)
+    Q, K = x["Q"].double().numpy(), x["K"].double().numpy()
+    NP, NB = z.shape[2:]
+    assert (NP, NB) == (3, 5)
+    for h in range(2):
+        S = idx[0, h]
+        for p in range(NP):
+            rows = range(256 * p, min(256 * p + 256, lk[0]))
+            if not len(rows):
+                assert np.all(np.isnan(z[0, h, p]))
+                continue
+            qb = np.mean([Q[0, S[i], h] for i in rows], axis=0)
+            for j in range(NB):
+                if j >= 2 * p:
+                    assert np.isnan(z[0, h, p, j])
+                    continue
+                kb = np.mean([K[0, S[i], 0] for i in range(128 * j, 128 * j + 128)], axis=0)
+                assert z[0, h, p, j] == pytest.approx(0.25 * qb @ kb, rel=1e-12, abs=1e-15)
+
+
+def test_block_select_rule_and_ties():
+    B, H, L = 1, 1, 1024                     # NP = 4, NB = 8
+    z = np.full((B, H, 4, 8), np.nan, np.float32)
+    z[0, 0, 3, :6] = [0.0, 5.0, 1.0, 4.0, 5.0, 2.0]      # max 5 (twice)
+    z[0, 0, 2, :4] = [3.0, 1.0, -1.0, 2.0]
+    z[0, 0, 1, :2] = [7.0, 0.0]
+    keep = oracle.block_select(z, np.array([L], np.int32), theta=1.0)
+    assert list(keep[0, 0, 3]) == [1, 1, 0, 1, 1, 0, 1, 1]   # 0, ties at 5, 4 >= 4, diag 6, 7
+    assert list(keep[0, 0, 2]) == [1, 0, 0, 1, 1, 1, 0, 0]   # 0, 2 >= 2, diag 4, 5
+    assert list(keep[0, 0, 1]) == [1, 0, 1, 1, 0, 0, 0, 0]   # 0, z1 = 0 < 6, diag 2, 3
+    assert list(keep[0, 0, 0]) == [1, 1, 0, 0, 0, 0, 0, 0]   # diag 0, 1
+    every = oracle.block_select(z, np.array([L], np.int32), theta=np.inf)
+    assert every[0, 0, 3, :8].sum() == 8
+    short = oracle.block_select(z, np.array([890], np.int32), theta=0.0)   # pair 3: no block 7
+    assert list(short[0, 0, 3]) == [1, 1, 0, 0, 1, 0, 1, 0]
+
+
+def test_block_attention_with_every_block_is_compressed_attention():
+    x, idx, lk = _block_case(L=700, keep=650, seed=3)
+    z = oracle.block_logits(x["Q"], x["K"], idx, lk)
+    keep = oracle.block_select(z.astype(np.float32), lk, theta=np.inf)
+    rows = [(0, h, i) for h in range(2) for i in (0, 1, 127, 128, 255, 256, 300, 511, 512, 649)]
+    got = oracle.attend_block_rows(x["Q"], x["K"], x["V"], idx, lk, keep, rows)
+    want = oracle.attend_rows(x["Q"], x["K"], x["V"], idx, lk, rows)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-14)
+
+
+def test_block_attention_matches_masked_softmax():
+    x, idx, lk = _block_case(L=640, keep=640, seed=4)
+    z = oracle.block_logits(x["Q"], x["K"], idx, lk)
+    keep = oracle.block_select(z.astype(np.float32), lk, theta=0.05)
+    assert keep.sum() < np.isfinite(z).sum() + 3 * 2 * 3      # something was dropped
+    Q, K, V = (x[k].double() for k in ("Q", "K", "V"))
+    for h in range(2):
+        S = torch.from_numpy(idx[0, h]).long()
+        q, k, v = Q[0, S, h], K[0, S, 0], V[0, S, 0]
+        logits = (q @ k.T) / np.sqrt(16)
+        allowed = torch.zeros(640, 640, dtype=torch.bool)
+        for i in range(640):
+            blocks = torch.from_numpy(keep[0, h, i // 256].astype(bool))
+            allowed[i, : i + 1] = blocks[torch.arange(i + 1) // 128]
+        ref = torch.softmax(logits.masked_fill(~allowed, float("-inf")), dim=1) @ v
+        rows = [(0, h, i) for i in range(0, 640, 7)]
+        got = oracle.attend_block_rows(x["Q"], x["K"], x["V"], idx, lk, keep, rows)
+        np.testing.assert_allclose(got, ref[::7].numpy(), rtol=0, atol=1e-13)
