@@ -29,6 +29,8 @@ METRIC = "token-sparse attn layer ms @128K Llama-8B shape; TFLOP/s & % roofline"
 STAGES = ("score", "budget", "select", "gather", "attn", "scatter")
 # fractions of the tokens pruned at 128K in the pages' own runs (L' = 0.456 L and 0.326 L)
 PAGES_SPARSITY = (0.544, 0.674)
+# thresholds of the block-sparse pattern (blocks within theta of a pair's best block mean)
+BLOCK_THETAS = (0.25, 0.1)
 
 
 def _peaks():
@@ -68,6 +70,27 @@ def l2_note(d) -> str:
             % (mb["Q"], mb["K"], mb["X"]) if big else
             "inputs not all larger than L2 (Q %.0f MB, K/V %.0f MB each, X %.0f MB); no flush"
             % (mb["Q"], mb["K"], mb["X"]))
+
+
+def block_useful_flops(mask, lk: int, d: int) -> float:
+    """Useful attention FLOPs (QK^T and PV, causal keys of kept blocks) of a block mask
+    [B=1, H, NP, NW] int32 for L' = lk: 4 d per visible (query, key) pair."""
+    import numpy as np
+    m = mask.cpu().numpy().view(np.uint32)[0]          # [H, NP, NW]
+    H, NP, NW = m.shape
+    bits = ((m[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(H, NP, NW * 32)
+    total = 0.0
+    for p in range((lk + 255) // 256):
+        kept = bits[:, p, :]                           # [H, NB]
+        for x in (0, 1):
+            r0 = 256 * p + 128 * x
+            rows = max(0, min(128, lk - r0))
+            if rows == 0:
+                continue
+            full = kept[:, : 2 * p + x].sum(axis=1) * 128.0       # blocks before the diagonal
+            diag = rows * (rows + 1) / 2.0                        # the tile's own block
+            total += float((full * rows + diag * kept[:, 2 * p + x]).sum())
+    return 4.0 * d * total
 
 
 def kv_union_rows(idx, lk: int, Hkv: int) -> int:
@@ -376,6 +399,42 @@ def run_ours(args, w, L, rank, world, local_rank):
         if tsa.tsa_get_device_status(ws) != 0:
             raise RuntimeError("device error in the pages'-sparsity runs")
 
+    # token + block composition: block-sparse attention inside the compressed space
+    blocks = None
+    if not args.no_pages_sparsity:
+        blocks = []
+        for th in BLOCK_THETAS:
+            for _ in range(2):
+                tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, ws=ws,
+                              block_theta=th)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+            for e in ev:
+                e.record(st)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            sync_all()
+            a.record(st)
+            for _ in range(2):
+                tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, ws=ws,
+                              block_theta=th, Lkeep=Lk, idx=idx, stage_events=ev)
+            b.record(st)
+            sync_all()
+            bms = job_max(a.elapsed_time(b) / 2, world, dev)
+            battn = ev[4].elapsed_time(ev[5])
+            Qh, Kh, _ = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk)
+            _, bmask = tsa.tsa_block_select(dm, Qh, Kh, Lk, th, logits=False)
+            del Qh, Kh
+            lkb = int(Lk.item())
+            useful = block_useful_flops(bmask, lkb, w.d)
+            blocks.append({"theta": th, "Lkeep": lkb, "layer_ms": bms,
+                           "attn_ms_incl_block_select": battn,
+                           "useful_fraction_of_compressed": useful / (2.0 * w.H * w.d * lkb * (lkb + 1)),
+                           "useful_attn_tflops": useful / (battn * 1e-3) / 1e12,
+                           "speedup_vs_dense_layer": (dense["layer_ms"] / bms) if dense else None})
+        torch.cuda.empty_cache()
+        if tsa.tsa_get_device_status(ws) != 0:
+            raise RuntimeError("device error in the block-sparse runs")
+
     # end to end through the public API with host buffers (copies inside the timed region)
     e2e = None
     if not args.no_e2e:
@@ -429,6 +488,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "overhead_fraction": 1.0 - attn_ms / sum(stage_ms.values()),
             "dense": dense,
             "pages_sparsity": pages,
+            "block_sparse": blocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk.summary(),

@@ -181,6 +181,34 @@ TSA_API tsa_status tsa_attn_gather(const tsa_dims *dims, const void *Q, const vo
                                    float scale, const void *X, void *Y, void *ws,
                                    size_t ws_bytes, void *stream);
 
+/* ---- Block-sparse attention inside the compressed space ---------------------------- */
+/* [notes] 关键发现 (token sparsity stacked on block-level sparsity is the most valuable
+ * pairing) and [blog] §3.2 ("token selection first, then block-sparse computation").
+ * The block choice is this library's own definition (the pages give none).  In head h's
+ * compressed order: query pair p = rows [256p, 256p + 256), key block j = rows
+ * [128j, 128j + 128), NP = ceil(L / 256) pairs, NB = ceil(L / 128) blocks of capacity.
+ *   logits[b,h,p,j] = scale * < mean of the pair's Qh rows, mean of block j's Kh rows >
+ *                     for j < 2p (NaN otherwise);
+ *   mask[b,h,p] (NW = ceil(NB / 32) uint32 words, bit j of word j / 32): block 0, the
+ *                     diagonal blocks 2p and 2p + 1 (if it exists), and every j < 2p with
+ *                     logits >= max_j logits - theta (one fp32 subtraction, fp32 compare).
+ * Means are fp32 sums in row order, dot products fp32 in a fixed order: deterministic.
+ * theta in [0, 3e38] (3e38 keeps every block).  logits [B,H,NP,NB] fp32 is optional
+ * (NULL: not written).  Qh, Kh as tsa_gather_qkv writes them.  ws:
+ * tsa_block_workspace_size() bytes. */
+TSA_API size_t tsa_block_workspace_size(const tsa_dims *dims);
+TSA_API tsa_status tsa_block_select(const tsa_dims *dims, const void *Qh, const void *Kh,
+                                    const int32_t *Lkeep, float scale, double theta,
+                                    float *logits, uint32_t *mask, void *ws, size_t ws_bytes,
+                                    void *stream);
+
+/* Compressed attention restricted to the kept blocks of `mask` (as tsa_block_select
+ * writes it): row i attends to the keys i' <= i whose block is kept for the pair of i.
+ * Otherwise as tsa_attn with dense == 0.  bf16 only. */
+TSA_API tsa_status tsa_attn_block(const tsa_dims *dims, const void *Qh, const void *Kh,
+                                  const void *Vh, const int32_t *Lkeep, const uint32_t *mask,
+                                  float scale, void *Oh, void *ws, size_t ws_bytes, void *stream);
+
 /* ---- Budget and score variants ([notes] 消融实验 and 关键设计 2) ------------------- */
 
 typedef enum { TSA_POOL_NONE = 0, TSA_POOL_MAX = 1, TSA_POOL_MEAN = 2 } tsa_pool_kind;
@@ -218,6 +246,9 @@ typedef struct {
     int32_t pool_width;    /* odd, 1..255 (ignored for POOL_NONE)  */
     int32_t direct_gather; /* 1: tsa_attn_gather instead of gather, attention, scatter
                               (bf16 only; same Y bit for bit)      */
+    double block_theta;    /* >= 0: block-sparse attention inside the compressed space with
+                              this theta (tsa_block_select, tsa_attn_block; bf16, staged
+                              path); negative or NaN: every block  */
 } tsa_layer_opts;
 
 /* tsa_layer with the budget and score variants of tsa_layer_opts (opts NULL: coverage

@@ -213,3 +213,90 @@ def test_attn_gather_reports_a_bad_index():
     ws = tsa.workspace(dm, 1)
     tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, d["X"], ws=ws)
     assert tsa.tsa_get_device_status(ws) == 1            # TSA_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- block-sparse attention
+def _keep_to_words(keep):
+    B, H, NP, NB = keep.shape
+    NW = (NB + 31) // 32
+    w = np.zeros((B, H, NP, NW), np.uint32)
+    for j in range(NB):
+        w[..., j // 32] |= (keep[..., j].astype(np.uint32) << np.uint32(j % 32))
+    return w
+
+
+def _compressed(B, L, H, Hkv, seed, keep):
+    x = make_inputs(B, L, H, Hkv, 128, torch.bfloat16, seed=seed)
+    d = {k: v.cuda() for k, v in x.items()}
+    dm = tsa.dims(d["Q"], d["K"])
+    s_h, _ = tsa.tsa_score(d["Q"], d["K"], 16)
+    Lk = torch.tensor(keep, dtype=torch.int32, device="cuda")
+    idx = tsa.tsa_select(dm, s_h, Lk)
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk)
+    return x, d, dm, Lk, idx, Qh, Kh, Vh
+
+
+@pytest.mark.parametrize("B,L,H,Hkv,keep,theta", [(1, 4096, 8, 2, [4096], 1.0),
+                                                  (2, 3000, 4, 4, [3000, 1111], 0.5),
+                                                  (1, 2600, 8, 2, [2555], 0.0)])
+def test_block_select_and_attention_match_oracle(B, L, H, Hkv, keep, theta):
+    x, d, dm, Lk, idx, Qh, Kh, Vh = _compressed(B, L, H, Hkv, seed=L + H, keep=keep)
+    z, mask = tsa.tsa_block_select(dm, Qh, Kh, Lk, theta)
+    zg = z.cpu().numpy()
+    ref = oracle.block_logits(x["Q"], x["K"], idx.cpu().numpy(), keep)
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(zg))
+    assert np.max(np.abs(zg[fin] - ref[fin])) <= 1e-4 * max(1.0, np.max(np.abs(ref[fin])))
+    want = _keep_to_words(oracle.block_select(zg, np.array(keep, np.int32), theta))
+    np.testing.assert_array_equal(mask.cpu().numpy().view(np.uint32), want)
+    Oh = tsa.tsa_attn_block(dm, Qh, Kh, Vh, Lk, mask)
+    keep_u8 = oracle.block_select(zg, np.array(keep, np.int32), theta)
+    rng = np.random.default_rng(0)
+    rows = [(b, h, int(i)) for b in range(B) for h in (0, H - 1)
+            for i in np.unique(np.concatenate([[0, 127, 128, 255, 256, keep[b] - 1],
+                                                 rng.integers(0, keep[b], 12)]))]
+    got = Oh.cpu().double().numpy()[tuple(np.asarray(rows).T)]
+    ref_o = oracle.attend_block_rows(x["Q"], x["K"], x["V"], idx.cpu().numpy(), keep, keep_u8, rows)
+    assert np.max(np.abs(got - ref_o)) <= 2e-2
+    if theta == 0.0:
+        assert keep_u8.sum() < sum(2 * ((k + 255) // 256) ** 2 for k in keep) * H  # sparse
+
+
+def test_block_theta_huge_equals_full_compressed_attention():
+    x, d, dm, Lk, idx, Qh, Kh, Vh = _compressed(1, 5000, 8, 2, seed=9, keep=[4800])
+    _, mask = tsa.tsa_block_select(dm, Qh, Kh, Lk, 3e38, logits=False)
+    assert torch.equal(tsa.tsa_attn_block(dm, Qh, Kh, Vh, Lk, mask), tsa.tsa_attn(dm, Qh, Kh, Vh, Lk))
+
+
+def test_layer_block_theta_equals_manual_chain():
+    x = make_inputs(1, 4096, 32, 8, 128, torch.bfloat16, seed=12)
+    d = {k: v.cuda() for k, v in x.items()}
+    dm = tsa.dims(d["Q"], d["K"])
+    Lk = torch.empty(1, dtype=torch.int32, device="cuda")
+    idx = torch.empty(1, 32, 4096, dtype=torch.int32, device="cuda")
+    Y = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, tau=0.01, Lkeep=Lk, idx=idx,
+                      block_theta=0.5)
+    Qh, Kh, Vh = tsa.tsa_gather_qkv(d["Q"], d["K"], d["V"], idx, Lk)
+    _, mask = tsa.tsa_block_select(dm, Qh, Kh, Lk, 0.5)
+    Oh = tsa.tsa_attn_block(dm, Qh, Kh, Vh, Lk, mask)
+    assert torch.equal(Y, tsa.tsa_scatter_residual(dm, Oh, idx, Lk, d["X"]))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_select_fp32_matches_oracle(d):
+    B, L, H, Hkv, keep, theta = 1, 1500, 4, 2, [1400], 0.3
+    x = make_inputs(B, L, H, Hkv, d, torch.float32, seed=d)
+    dd = {k: v.cuda() for k, v in x.items()}
+    dm = tsa.dims(dd["Q"], dd["K"])
+    s_h, _ = tsa.tsa_score(dd["Q"], dd["K"], 16)
+    Lk = torch.tensor(keep, dtype=torch.int32, device="cuda")
+    idx = tsa.tsa_select(dm, s_h, Lk)
+    Qh, Kh, _ = tsa.tsa_gather_qkv(dd["Q"], dd["K"], dd["V"], idx, Lk)
+    z, mask = tsa.tsa_block_select(dm, Qh, Kh, Lk, theta)
+    zg = z.cpu().numpy()
+    ref = oracle.block_logits(x["Q"], x["K"], idx.cpu().numpy(), keep)
+    fin = np.isfinite(ref)
+    assert np.array_equal(fin, np.isfinite(zg))
+    assert np.max(np.abs(zg[fin] - ref[fin])) <= 1e-5 * max(1.0, np.max(np.abs(ref[fin])))
+    want = _keep_to_words(oracle.block_select(zg, np.array(keep, np.int32), theta))
+    np.testing.assert_array_equal(mask.cpu().numpy().view(np.uint32), want)

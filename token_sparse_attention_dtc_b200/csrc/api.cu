@@ -19,6 +19,10 @@ cudaError_t launch_score_tc(const tsa_dims &, const void *, const void *, int, f
                             const WsLayout &, char *, cudaStream_t, uint32_t);
 cudaError_t launch_fill_lkeep(int, int32_t, int32_t *, cudaStream_t);
 size_t drift_workspace_bytes(int, long long);
+size_t block_scratch_bytes(const tsa_dims &);
+size_t block_mask_words(const tsa_dims &);
+cudaError_t launch_block_select(const tsa_dims &, const void *, const void *, const int32_t *,
+                                float, float, float *, uint32_t *, char *, cudaStream_t);
 cudaError_t launch_attn_gather(const tsa_dims &, const void *, const void *, const void *,
                                const int32_t *, const int32_t *, float, const void *, void *,
                                Control *, cudaStream_t, uint32_t);
@@ -40,7 +44,7 @@ cudaError_t launch_attn_simt(const tsa_dims &, const void *, const void *, const
                              const int32_t *, int, float, void *, cudaStream_t);
 cudaError_t launch_attn_tc(const tsa_dims &, const void *, const void *, const void *,
                            const int32_t *, int, float, void *, Control *, cudaStream_t,
-                           uint32_t);
+                           uint32_t, const uint32_t * = nullptr);
 cudaError_t launch_scatter(const tsa_dims &, const void *, const int32_t *, const int32_t *,
                            const void *, void *, cudaStream_t);
 
@@ -136,7 +140,7 @@ WsLayout ws_layout(const tsa_dims &dm, int q) {
 }
 
 struct LayerLayout {
-    size_t s_h, s_hp, s_l, lkeep, idx, qh, kh, vh, oh, total;
+    size_t s_h, s_hp, s_l, lkeep, idx, blk_scratch, blk_mask, qh, kh, vh, oh, total;
 };
 
 static LayerLayout layer_layout(const tsa_dims &dm, int q) {
@@ -148,6 +152,8 @@ static LayerLayout layer_layout(const tsa_dims &dm, int q) {
     y.s_l = off; off = align256(off + 4 * (size_t)dm.B * dm.L);
     y.lkeep = off; off = align256(off + 4 * (size_t)dm.B);
     y.idx = off; off = align256(off + 4 * BHL);
+    y.blk_scratch = off; off = align256(off + block_scratch_bytes(dm));  // block-sparse means
+    y.blk_mask = off; off = align256(off + 4 * block_mask_words(dm));
     const size_t t = align256(BHL * dm.d * esize(dm));
     y.qh = off; off += t;
     y.kh = off; off += t;
@@ -182,11 +188,11 @@ static tsa_status do_score(const tsa_dims &dm, const void *Q, const void *K, int
 
 static tsa_status do_attn(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                           const int32_t *Lkeep, int dense, float scale, void *O, char *ws,
-                          cudaStream_t st) {
+                          cudaStream_t st, const uint32_t *bmask = nullptr) {
     cudaError_t e;
     if (dm.dtype == TSA_BF16)
         e = launch_attn_tc(dm, Q, K, V, Lkeep, dense, scale, O, reinterpret_cast<Control *>(ws),
-                           st, g_wait_limit_us);
+                           st, g_wait_limit_us, bmask);
     else
         e = launch_attn_simt(dm, Q, K, V, Lkeep, dense, scale, O, st);
     return cuda_status(e, "tsa_attn");
@@ -347,6 +353,51 @@ static tsa_status do_attn_gather(const tsa_dims &dm, const void *Q, const void *
                        "tsa_attn_gather");
 }
 
+size_t tsa_block_workspace_size(const tsa_dims *dims) {
+    if (check_dims(dims) != TSA_OK) return 0;
+    return block_scratch_bytes(*dims);
+}
+
+static tsa_status check_theta(double theta) {
+    if (!(theta >= 0.0 && theta <= 3.0e38))
+        return fail(TSA_ERR_INVALID_ARG, "theta must be in [0, 3e38] (use 3e38 for every block)");
+    return TSA_OK;
+}
+
+tsa_status tsa_block_select(const tsa_dims *dims, const void *Qh, const void *Kh,
+                            const int32_t *Lkeep, float scale, double theta, float *logits,
+                            uint32_t *mask, void *ws, size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_theta(theta));
+    TSA_TRY(check_ptr(Qh, "Qh"));
+    TSA_TRY(check_ptr(Kh, "Kh"));
+    TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    TSA_TRY(check_ptr(mask, "mask"));
+    if (logits) TSA_TRY(check_ptr(logits, "logits"));
+    TSA_TRY(check_ws(ws, ws_bytes, block_scratch_bytes(*dims)));
+    return cuda_status(launch_block_select(*dims, Qh, Kh, Lkeep, scale, (float)theta, logits, mask,
+                                           (char *)ws, (cudaStream_t)stream),
+                       "tsa_block_select");
+}
+
+tsa_status tsa_attn_block(const tsa_dims *dims, const void *Qh, const void *Kh, const void *Vh,
+                          const int32_t *Lkeep, const uint32_t *mask, float scale, void *Oh,
+                          void *ws, size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    if (dims->dtype != TSA_BF16)
+        return fail(TSA_ERR_UNSUPPORTED, "block-sparse attention runs the bf16 tensor-core path only");
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_ptr(Qh, "Qh"));
+    TSA_TRY(check_ptr(Kh, "Kh"));
+    TSA_TRY(check_ptr(Vh, "Vh"));
+    TSA_TRY(check_ptr(Lkeep, "Lkeep"));
+    TSA_TRY(check_ptr(mask, "mask"));
+    TSA_TRY(check_ptr(Oh, "Oh"));
+    TSA_TRY(check_ws(ws, ws_bytes, sizeof(Control)));
+    return do_attn(*dims, Qh, Kh, Vh, Lkeep, 0, scale, Oh, (char *)ws, (cudaStream_t)stream, mask);
+}
+
 tsa_status tsa_attn_gather(const tsa_dims *dims, const void *Q, const void *K, const void *V,
                            const int32_t *idx, const int32_t *Lkeep, float scale, const void *X,
                            void *Y, void *ws, size_t ws_bytes, void *stream) {
@@ -383,6 +434,12 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
     if (o.pool != TSA_POOL_NONE) TSA_TRY(check_pool(o.pool, o.pool_width));
     if (o.direct_gather && dims->dtype != TSA_BF16)
         return fail(TSA_ERR_UNSUPPORTED, "direct gather runs the bf16 tensor-core path only");
+    const bool blocks = o.block_theta >= 0.0;  // NaN or negative: every block
+    if (blocks) {
+        TSA_TRY(check_theta(o.block_theta));
+        if (dims->dtype != TSA_BF16 || o.direct_gather)
+            return fail(TSA_ERR_UNSUPPORTED, "block sparsity runs the bf16 staged path only");
+    }
     TSA_TRY(check_ptr(Q, "Q"));
     TSA_TRY(check_ptr(K, "K"));
     TSA_TRY(check_ptr(V, "V"));
@@ -441,7 +498,14 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
     TSA_TRY(cuda_status(launch_gather(dm, Q, K, V, idx, Lk, Qh, Kh, Vh, (Control *)w, st),
                         "tsa_layer gather"));
     TSA_TRY(rec(4));
-    TSA_TRY(do_attn(dm, Qh, Kh, Vh, Lk, 0, scale, Oh, w, st));
+    uint32_t *bm = nullptr;
+    if (blocks) {  // block-sparse pattern of the compressed problem (part of the attention)
+        bm = (uint32_t *)(w + y.blk_mask);
+        TSA_TRY(cuda_status(launch_block_select(dm, Qh, Kh, Lk, scale, (float)o.block_theta,
+                                                nullptr, bm, w + y.blk_scratch, st),
+                            "tsa_layer block select"));
+    }
+    TSA_TRY(do_attn(dm, Qh, Kh, Vh, Lk, 0, scale, Oh, w, st, bm));
     TSA_TRY(rec(5));
     TSA_TRY(cuda_status(launch_scatter(dm, Oh, idx, Lk, X, Y, st), "tsa_layer scatter"));
     return rec(6);
@@ -452,7 +516,7 @@ tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const v
                      float scale, float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
                      int32_t *idx_out, void *ws, size_t ws_bytes, void *stream,
                      void *const *stage_events) {
-    tsa_layer_opts o{TSA_BUDGET_COVERAGE, tau, 0.0, TSA_POOL_NONE, 1, 0};
+    tsa_layer_opts o{TSA_BUDGET_COVERAGE, tau, 0.0, TSA_POOL_NONE, 1, 0, -1.0};
     return layer_impl(dims, Q, K, V, X, Y, is_sparse, q, o, scale, s_h_out, s_l_out, Lkeep_out,
                       idx_out, ws, ws_bytes, stream, stage_events);
 }
@@ -463,7 +527,8 @@ tsa_status tsa_layer_ex(const tsa_dims *dims, const void *Q, const void *K, cons
                         float *s_l_out, int32_t *Lkeep_out, int32_t *idx_out, void *ws,
                         size_t ws_bytes, void *stream, void *const *stage_events) {
     const tsa_layer_opts o = opts ? *opts
-                                  : tsa_layer_opts{TSA_BUDGET_COVERAGE, 0.005, 0.0, TSA_POOL_NONE, 1, 0};
+                                  : tsa_layer_opts{TSA_BUDGET_COVERAGE, 0.005, 0.0, TSA_POOL_NONE, 1, 0,
+                                                   -1.0};
     return layer_impl(dims, Q, K, V, X, Y, is_sparse, q, o, scale, s_h_out, s_l_out, Lkeep_out,
                       idx_out, ws, ws_bytes, stream, stage_events);
 }

@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ Lkeep, int dense,
           int L, int H, int Hkv, float sl2, __nv_bfloat16 *__restrict__ O, GatherArgs ga,
-          Control *ctl, uint64_t limit_ns, int stall) {
+          const uint32_t *__restrict__ bmask, Control *ctl, uint64_t limit_ns, int stall) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem<D> &sm = *reinterpret_cast<AttnSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -273,7 +273,22 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int i0 = pair * 2 * kBM;  // first row of tile A
     if (i0 >= Lk) return;
     const bool hasB = i0 + kBM < Lk;
-    const int nA = 2 * pair + 1, nB = hasB ? 2 * pair + 2 : 0;
+    // Key blocks of this pair: all of 0..2p+1, or the kept ones of the block-sparse mask
+    // (ascending; block 0 and the diagonal blocks 2p, 2p+1 are always kept).
+    const int NW = ceil_div(ceil_div(L, kBN), 32);
+    const uint32_t *bm = bmask ? bmask + ((size_t)bh * npairs + pair) * NW : nullptr;
+    int nA = 2 * pair + 1, nB = hasB ? 2 * pair + 2 : 0;
+    if (bm) {
+        int below = 0, all = 0;  // kept blocks <= 2p, and in total
+        for (int w = 0; w < NW; ++w) {
+            const uint32_t word = __ldg(bm + w);
+            all += __popc(word);
+            const int lo = 2 * pair + 1 - 32 * w;  // bits [0, lo) of this word are <= 2p
+            below += __popc(lo >= 32 ? word : (lo > 0 ? word & ((1u << lo) - 1u) : 0u));
+        }
+        nA = below;
+        nB = hasB ? all : 0;
+    }
     const int nkv = hasB ? nB : nA;
     const int kvh = (dense || kGather) ? h / (H / Hkv) : h;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -314,6 +329,15 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     } else if (warp == 0) {
         if (lane == 0) {
             int issued = 0;  // K/V tiles issued (negative: K of tile -issued-1 only)
+            int cw = 0;      // block-sparse: current mask word and its unvisited bits
+            uint32_t cur = bm ? __ldg(bm) : 0u;
+            auto next_block = [&](int j) -> int {
+                if (!bm) return j;
+                while (cur == 0u) cur = __ldg(bm + (++cw));
+                const int e = __ffs(cur) - 1;
+                cur &= cur - 1u;
+                return cw * 32 + e;
+            };
             mbar_expect_tx(&sm.q_full, 2 * TILE);
 #pragma unroll
             for (int x = 0; x < 2; ++x)
@@ -324,11 +348,12 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % kStages;
                 const uint32_t ph = ((j / kStages) & 1) ^ 1;
+                const int kb = next_block(j);  // key block of step j
                 if (!(ok = mbar_wait(&sm.k_empty[s], ph, limit_ns, abort))) break;
                 mbar_expect_tx(&sm.k_full[s], TILE);
 #pragma unroll
                 for (int db = 0; db < NDB; ++db)
-                    tma_load_4d(sm.k[s] + db * kBN * 128, &tmK, &sm.k_full[s], db * 64, j * kBN,
+                    tma_load_4d(sm.k[s] + db * kBN * 128, &tmK, &sm.k_full[s], db * 64, kb * kBN,
                                 kvh, b);
                 if (!(ok = mbar_wait(&sm.v_empty[s], ph, limit_ns, abort))) {
                     issued = -(j + 1);
@@ -337,7 +362,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 mbar_expect_tx(&sm.v_full[s], TILE);
 #pragma unroll
                 for (int db = 0; db < NDB; ++db)
-                    tma_load_4d(sm.v[s] + db * kBN * 128, &tmV, &sm.v_full[s], db * 64, j * kBN,
+                    tma_load_4d(sm.v[s] + db * kBN * 128, &tmV, &sm.v_full[s], db * 64, kb * kBN,
                                 kvh, b);
                 issued = j + 1;
             }
@@ -503,8 +528,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 template <int D, bool kGather>
 static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                                 const int32_t *Lkeep, int dense, float scale, void *O,
-                                const GatherArgs &ga, Control *ctl, cudaStream_t st,
-                                uint32_t limit_us) {
+                                const GatherArgs &ga, const uint32_t *bmask, Control *ctl,
+                                cudaStream_t st, uint32_t limit_us) {
     CUtensorMap tq, tk, tv;
     memset(&tq, 0, sizeof tq);  // the direct-gather mode reads no tensor map
     memset(&tk, 0, sizeof tk);
@@ -534,19 +559,19 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
     const long nblocks = (long)ceil_div(dm.L, 2 * kBM) * dm.B * dm.H;
     k_attn_tc<D, kGather><<<(unsigned)nblocks, kThreads, smem, st>>>(
         tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
-        (__nv_bfloat16 *)O, ga, ctl, (uint64_t)limit_us * 1000ull, test_stall());
+        (__nv_bfloat16 *)O, ga, bmask, ctl, (uint64_t)limit_us * 1000ull, test_stall());
     note_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attn_tc(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                            const int32_t *Lkeep, int dense, float scale, void *O, Control *ctl,
-                           cudaStream_t st, uint32_t limit_us) {
+                           cudaStream_t st, uint32_t limit_us, const uint32_t *bmask) {
     const GatherArgs none{};
-    return dm.d == 64
-               ? attn_tc_impl<64, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, ctl, st, limit_us)
-               : attn_tc_impl<128, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, ctl, st,
-                                          limit_us);
+    return dm.d == 64 ? attn_tc_impl<64, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, bmask,
+                                                ctl, st, limit_us)
+                      : attn_tc_impl<128, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, bmask,
+                                                 ctl, st, limit_us);
 }
 
 // Compressed attention reading Q, K, V rows through idx, with Y = X + Ô written into the
@@ -563,8 +588,9 @@ cudaError_t launch_attn_gather(const tsa_dims &dm, const void *Q, const void *K,
     ga.X = (const __nv_bfloat16 *)X;
     ga.Y = (__nv_bfloat16 *)Y;
     return dm.d == 64
-               ? attn_tc_impl<64, true>(dm, Q, K, V, Lkeep, 0, scale, nullptr, ga, ctl, st, limit_us)
-               : attn_tc_impl<128, true>(dm, Q, K, V, Lkeep, 0, scale, nullptr, ga, ctl, st,
+               ? attn_tc_impl<64, true>(dm, Q, K, V, Lkeep, 0, scale, nullptr, ga, nullptr, ctl, st,
+                                        limit_us)
+               : attn_tc_impl<128, true>(dm, Q, K, V, Lkeep, 0, scale, nullptr, ga, nullptr, ctl, st,
                                          limit_us);
 }
 

@@ -25,7 +25,8 @@ EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_b
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
            "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall",
            "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex",
-           "tsa_drift_workspace_size", "tsa_drift", "tsa_attn_gather")
+           "tsa_drift_workspace_size", "tsa_drift", "tsa_attn_gather",
+           "tsa_block_workspace_size", "tsa_block_select", "tsa_attn_block")
 POOL_NONE, POOL_MAX, POOL_MEAN = 0, 1, 2
 BUDGET_COVERAGE, BUDGET_FIXED = 0, 1
 
@@ -45,7 +46,8 @@ class LayerOpts(ctypes.Structure):
     """tsa_layer_opts of include/tsa.h."""
     _fields_ = [("budget", ctypes.c_int32), ("tau", ctypes.c_double),
                 ("sparsity", ctypes.c_double), ("pool", ctypes.c_int32),
-                ("pool_width", ctypes.c_int32), ("direct_gather", ctypes.c_int32)]
+                ("pool_width", ctypes.c_int32), ("direct_gather", ctypes.c_int32),
+                ("block_theta", ctypes.c_double)]
 
 
 def lib():
@@ -77,6 +79,9 @@ def lib():
             "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
             "tsa_budget_fixed": (I32, [DP, D, P, P]),
             "tsa_attn_gather": (I32, [DP, P, P, P, P, P, F, P, P, P, SZ, P]),
+            "tsa_block_workspace_size": (SZ, [DP]),
+            "tsa_block_select": (I32, [DP, P, P, P, F, D, P, P, P, SZ, P]),
+            "tsa_attn_block": (I32, [DP, P, P, P, P, P, F, P, P, SZ, P]),
             "tsa_drift_workspace_size": (SZ, [I32, ctypes.c_int64]),
             "tsa_drift": (I32, [I32, ctypes.c_int64, I32, I32, P, D, D, P, P, P, SZ, P]),
             "tsa_pool_scores": (I32, [DP, P, I32, I32, P, P, P, SZ, P]),
@@ -262,6 +267,42 @@ def tsa_attn_gather(Q, K, V, idx, Lkeep, X, Y=None, scale: float | None = None, 
     return Y
 
 
+def block_shape(dm: Dims):
+    """(NP, NB, NW) of the block-sparse pattern for these dims."""
+    NP, NB = (dm.L + 255) // 256, (dm.L + 127) // 128
+    return NP, NB, (NB + 31) // 32
+
+
+def tsa_block_select(dm: Dims, Qh, Kh, Lkeep, theta: float, scale: float | None = None,
+                     logits: bool = True, ws=None, stream=None):
+    """Block logits [B, H, NP, NB] (or None) and kept-block mask [B, H, NP, NW] uint32."""
+    _need_cuda(Qh, Kh, Lkeep)
+    NP, NB, NW = block_shape(dm)
+    z = torch.empty(dm.B, dm.H, NP, NB, dtype=torch.float32, device=Qh.device) if logits else None
+    mask = torch.empty(dm.B, dm.H, NP, NW, dtype=torch.int32, device=Qh.device)
+    if ws is None:
+        ws = torch.zeros(max(256, lib().tsa_block_workspace_size(ctypes.byref(dm))),
+                         dtype=torch.uint8, device=Qh.device)
+    _check(lib().tsa_block_select(ctypes.byref(dm), _p(Qh), _p(Kh), _p(Lkeep),
+                                  default_scale(dm.d) if scale is None else scale, float(theta),
+                                  _p(z), _p(mask), _p(ws), ws.numel(), _stream(stream)))
+    return z, mask
+
+
+def tsa_attn_block(dm: Dims, Qh, Kh, Vh, Lkeep, mask, scale: float | None = None, Oh=None,
+                   ws=None, stream=None):
+    """Compressed attention restricted to the kept blocks of mask."""
+    _need_cuda(Qh, Kh, Vh, Lkeep, mask)
+    if Oh is None:
+        Oh = torch.empty_like(Qh)
+    if ws is None:
+        ws = workspace(dm, 1, device=Qh.device)
+    _check(lib().tsa_attn_block(ctypes.byref(dm), _p(Qh), _p(Kh), _p(Vh), _p(Lkeep), _p(mask),
+                                default_scale(dm.d) if scale is None else scale, _p(Oh), _p(ws),
+                                ws.numel(), _stream(stream)))
+    return Oh
+
+
 def tsa_budget_fixed(dm: Dims, sparsity: float, Lkeep=None, device=None, stream=None):
     """Fixed-ratio budget: Lkeep[b] = L - floor(sparsity * L)."""
     if Lkeep is None:
@@ -289,7 +330,8 @@ def tsa_pool_scores(dm: Dims, s_h, kind: int, width: int, s_h_out=None, s_l_out=
 def tsa_layer(Q, K, V, X, Y=None, is_sparse: bool = True, q: int = 16, tau: float = 0.005,
               scale: float | None = None, s_h=None, s_l=None, Lkeep=None, idx=None, ws=None,
               stream=None, stage_events=None, sparsity: float | None = None,
-              pool: int = POOL_NONE, pool_width: int = 1, direct: bool = False):
+              pool: int = POOL_NONE, pool_width: int = 1, direct: bool = False,
+              block_theta: float | None = None):
     """One Token Sparse Attention layer: returns Y = X + Decompress(Ô) (or the dense layer).
     sparsity (fixed-ratio budget instead of tau) and pool / pool_width (pooled head
     scores) and direct (fused compress + attention + decompress) select the variants of
@@ -304,14 +346,14 @@ def tsa_layer(Q, K, V, X, Y=None, is_sparse: bool = True, q: int = 16, tau: floa
     if stage_events is not None:
         ev = (ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
     sc = default_scale(dm.d) if scale is None else scale
-    if sparsity is None and pool == POOL_NONE and not direct:
+    if sparsity is None and pool == POOL_NONE and not direct and block_theta is None:
         _check(lib().tsa_layer(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y),
                                int(is_sparse), q, float(tau), sc, _p(s_h), _p(s_l), _p(Lkeep),
                                _p(idx), _p(ws), ws.numel(), _stream(stream), ev))
         return Y
     o = LayerOpts(BUDGET_COVERAGE if sparsity is None else BUDGET_FIXED, float(tau),
                   0.0 if sparsity is None else float(sparsity), int(pool), int(pool_width),
-                  int(bool(direct)))
+                  int(bool(direct)), -1.0 if block_theta is None else float(block_theta))
     _check(lib().tsa_layer_ex(ctypes.byref(dm), _p(Q), _p(K), _p(V), _p(X), _p(Y),
                               int(is_sparse), q, ctypes.byref(o), sc, _p(s_h), _p(s_l),
                               _p(Lkeep), _p(idx), _p(ws), ws.numel(), _stream(stream), ev))
