@@ -401,7 +401,7 @@ def run_ours(args, w, L, rank, world, local_rank):
 
     # token + block composition: block-sparse attention inside the compressed space
     blocks = None
-    if not args.no_pages_sparsity:
+    if not args.no_pages_sparsity and w.dtype == torch.bfloat16:  # tcgen05 path only
         blocks = []
         for th in BLOCK_THETAS:
             for _ in range(2):
