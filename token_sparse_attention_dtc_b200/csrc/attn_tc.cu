@@ -155,12 +155,6 @@ __device__ __forceinline__ bool gather_producer(AttnSmem<D> &sm, const GatherArg
     return ok;
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
 // P = 2^(S*sl2 - mu) of one row, packed to bf16x2 over sr[0..63]; returns the row sum of
 // the fp32 values.  Paired fp32 instructions for the scale-subtract and the sums.
 // kDiag: the diagonal tile, whose masked entries are -inf and give exactly 0.  (The two

@@ -44,9 +44,9 @@ template <int D> struct ScoreSmem {
     static constexpr int KT = kTile * D * 2;  // bytes of one K tile
     alignas(1024) uint8_t q[2 * 128 * D * 2];  // up to 256 query rows, swizzled, K-major
     alignas(1024) uint8_t k[kStages][KT];
-    uint64_t k_full[kStages], k_empty[kStages], acc_full[2], acc_empty[2], drain;
+    uint64_t k_full[kStages], k_empty[kStages], acc_full[4], acc_empty[4], drain;
     uint64_t stall;     // test hook: initialised, never completed
-    float2 stat[256];   // pass 2: (max, 1/sum) per query row
+    alignas(16) float mlog[256];  // pass 2: max + log2(sum) per query row (log2 units)
     float2 red[4][256]; // pass 1: per column group (max, sum) per query row
     uint32_t tmem_base;
     int abort, never, gbar_ok;
@@ -100,6 +100,10 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
     const int split = blockIdx.x, bg = group0 + blockIdx.y;
     const int b = bg / Hkv, kv = bg % Hkv, G = H / Hkv, N = G * qe;
     const int RB = (N + 127) / 128;   // pass 1 row blocks
+    // TMEM accumulator ring: 4 buffers of 128 columns when one row block (and <= 128
+    // query columns in pass 2) suffices, else 2 of 256; the MMA runs nbuf - 1 tiles ahead.
+    const int lgb = RB == 1 ? 2 : 1, nbuf = 1 << lgb;
+    const uint32_t bstride = 512u >> lgb;
     const int Npad = (N + 15) & ~15;  // pass 2 MMA N
     const int nrows = RB * 128;       // query rows held in shared memory
     const int ntiles = (L + kTile - 1) / kTile;
@@ -114,7 +118,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
             mbar_init(&sm.k_full[s], 1);
             mbar_init(&sm.k_empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < 4; ++a) {
             mbar_init(&sm.acc_full[a], 1);
             mbar_init(&sm.acc_empty[a], kEpiWarps * 32);
         }
@@ -166,13 +170,13 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
             // Test hook: a wait that nothing completes, so it runs out after limit_ns.
             if (stall) ok = mbar_wait(&sm.stall, 0, limit_ns, abort);
             for (int it = 0; it < total && ok; ++it) {
-                const int s = it % kStages, a = it & 1;
+                const int s = it % kStages, a = it & (nbuf - 1);
                 if (!(ok = mbar_wait(&sm.k_full[s], (it / kStages) & 1, limit_ns, abort))) break;
-                if (!(ok = mbar_wait(&sm.acc_empty[a], ((it >> 1) & 1) ^ 1, limit_ns, abort)))
+                if (!(ok = mbar_wait(&sm.acc_empty[a], ((it >> lgb) & 1) ^ 1, limit_ns, abort)))
                     break;
                 tc_fence_after();
                 const uint32_t ka = smem_u32(sm.k[s]);
-                const uint32_t dacc = tmem + a * 256;
+                const uint32_t dacc = tmem + a * bstride;
                 if (it < count) {
                     for (int rb = 0; rb < RB; ++rb)
 #pragma unroll
@@ -217,8 +221,8 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                 pr[rb] = n < N ? L - qe + (n % qe) : -1;  // -1: padding row, never valid
             }
             for (int it = 0; it < count; ++it) {
-                const int a = it & 1;
-                ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
+                const int a = it & (nbuf - 1);
+                ok = mbar_wait(&sm.acc_full[a], (it >> lgb) & 1, limit_ns, abort);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
                 const int tc0 = tile_at(it) * kTile + cg * 32;  // token of column 0 here
@@ -226,30 +230,47 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                 for (int rb = 0; rb < RB; ++rb) {
                     if (rb * 128 + wq * 32 >= N) continue;  // whole warp on padding rows
                     uint32_t v[32];
-                    tmem_ld32(tmem + a * 256 + rb * 128 + cg * 32 + lo, v);
+                    tmem_ld32(tmem + a * bstride + rb * 128 + cg * 32 + lo, v);
                     tmem_ld_wait();
                     if (pr[rb] < 0) continue;
-                    float cm = -INFINITY;
+                    float cm;
+                    if (!tail) {  // every token here precedes every recent query
+                        float c0 = __uint_as_float(v[0]), c1 = __uint_as_float(v[1]);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        float z = __uint_as_float(v[e]);
-                        if (tail && tc0 + e > pr[rb]) z = -INFINITY;
-                        v[e] = __float_as_uint(z);
-                        cm = fmaxf(cm, z);
+                        for (int e = 2; e < 30; e += 4) {
+                            c0 = fmax3(c0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                            c1 = fmax3(c1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                        }
+                        cm = fmax3(c0, c1, fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31])));
+                    } else {
+                        cm = -INFINITY;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            float z = __uint_as_float(v[e]);
+                            if (tc0 + e > pr[rb]) z = -INFINITY;
+                            v[e] = __float_as_uint(z);
+                            cm = fmaxf(cm, z);
+                        }
+                        if (cm == -INFINITY) continue;
                     }
-                    if (cm == -INFINITY) continue;
                     cm *= sl2;
                     if (cm > m[rb]) {
                         l[rb] = (m[rb] == -INFINITY) ? 0.0f : l[rb] * ex2(m[rb] - cm);
                         m[rb] = cm;
                     }
-                    float a0 = 0.0f, a1 = 0.0f;
+                    const float nm = -m[rb];
+                    float a0 = 0.0f, a1 = 0.0f, b0 = 0.0f, b1 = 0.0f;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        a0 += ex2(fmaf(__uint_as_float(v[e]), sl2, -m[rb]));
-                        a1 += ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -m[rb]));
+                    for (int e = 0; e < 32; e += 4) {  // paired fp32: two columns per FMA / add
+                        float x0, x1, x2, x3;
+                        fma2(x0, x1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), sl2, sl2,
+                             nm, nm);
+                        fma2(x2, x3, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), sl2,
+                             sl2, nm, nm);
+                        add2(a0, a1, a0, a1, ex2(x0), ex2(x1));
+                        add2(b0, b1, b0, b1, ex2(x2), ex2(x3));
                     }
-                    l[rb] += a0 + a1;
+                    l[rb] += (a0 + a1) + (b0 + b1);
                 }
                 tc_fence_before();
                 mbar_arrive(&sm.acc_empty[a]);
@@ -294,33 +315,49 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                 const float2 p = __ldcg(&part[((size_t)bg * nsplit + s) * N + et]);
                 online_merge(mm, ll, p.x, p.y);
             }
-            sm.stat[et] = make_float2(mm, 1.0f / ll);
+            sm.mlog[et] = mm + log2f(ll);  // exp2(z - m) / l = exp2(z - (m + log2 l))
         }
         named_barrier(1, kEpiWarps * 32);
         // ---- pass 2: thread owns token r of the tile and the heads g = cg, cg + 4, ...;
         // head g's query rows are the columns [g*qe, (g+1)*qe), summed in row order.
         for (int it = count; it < total && ok; ++it) {
-            const int a = it & 1;
-            ok = mbar_wait(&sm.acc_full[a], (it >> 1) & 1, limit_ns, abort);
+            const int a = it & (nbuf - 1);
+            ok = mbar_wait(&sm.acc_full[a], (it >> lgb) & 1, limit_ns, abort);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
             const int t = tile_at(it) * kTile + r;
+            const bool early = tile_at(it) * kTile + kTile - 1 <= pmin;  // no query follows
             for (int g = cg; g < G; g += 4) {
                 const int c0 = g * qe, c1 = c0 + qe;
-                float acc = 0.0f;
+                float acc = 0.0f, a0 = 0.0f, a1 = 0.0f;
                 for (int cs = c0 & ~15; cs < c1; cs += 16) {
                     uint32_t v[16];
-                    tmem_ld16(tmem + a * 256 + cs + lo, v);
+                    tmem_ld16(tmem + a * bstride + cs + lo, v);
                     tmem_ld_wait();
+                    if (early && cs >= c0 && cs + 16 <= c1) {  // all 16 columns count
+                        const float4 *ml = reinterpret_cast<const float4 *>(sm.mlog + cs);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int n = cs + e;
-                        if (n < c0 || n >= c1) continue;
-                        const float2 st = sm.stat[n];
-                        if (t <= pmin + (n - c0))
-                            acc = fmaf(ex2(fmaf(__uint_as_float(v[e]), sl2, -st.x)), st.y, acc);
+                        for (int e = 0; e < 16; e += 4) {
+                            const float4 mq = ml[e / 4];
+                            float x0, x1, x2, x3;
+                            fma2(x0, x1, __uint_as_float(v[e]), __uint_as_float(v[e + 1]), sl2,
+                                 sl2, -mq.x, -mq.y);
+                            fma2(x2, x3, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]), sl2,
+                                 sl2, -mq.z, -mq.w);
+                            add2(a0, a1, a0, a1, ex2(x0), ex2(x1));
+                            add2(a0, a1, a0, a1, ex2(x2), ex2(x3));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int n = cs + e;
+                            if (n < c0 || n >= c1) continue;
+                            if (t <= pmin + (n - c0))
+                                acc += ex2(fmaf(__uint_as_float(v[e]), sl2, -sm.mlog[n]));
+                        }
                     }
                 }
+                acc += a0 + a1;
                 if (t < L) s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
             }
             tc_fence_before();

@@ -220,6 +220,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return w;
 }
 
+// Three-input fp32 maximum.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // ---------------------------------------------------------------- paired fp32 ---
 // sm_100a executes two fp32 adds or FMAs per instruction on register pairs; each lane
 // of the pair rounds exactly like the scalar instruction (round to nearest even).
