@@ -367,6 +367,34 @@ def run_ours(args, w, L, rank, world, local_rank):
                  "attn_frac_of_sustained": dflops / (dattn * 1e-3) / 1e12 / peaks["bf16_sus"],
                  "speedup_sparse_vs_dense_layer": dms / ms_step}
 
+    # the same layer captured once in a CUDA graph and replayed (no host launch gaps)
+    graph = None
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(st)
+        with torch.cuda.stream(side):
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk,
+                          idx=idx, ws=ws)
+        st.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk,
+                          idx=idx, ws=ws)
+        g.replay()
+        sync_all()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(args.steps):
+            g.replay()
+        b.record(st)
+        sync_all()
+        graph = {"layer_ms": job_max(a.elapsed_time(b) / args.steps, world, dev) / world}
+        del g
+    except Exception as e:  # reported, not required
+        graph = {"error": str(e).splitlines()[0][:200]}
+
     # the whole layer at the pages' sparsities (54.4% and 67.4% of the tokens pruned at
     # 128K), through the fixed-ratio budget on the same synthetic inputs
     pages = None
@@ -513,6 +541,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "layer_tflops": flops / (ms_step * 1e-3) / 1e12,
             "overhead_fraction": 1.0 - attn_ms / sum(stage_ms.values()),
             "dense": dense,
+            "graph_replay": graph,
             "pages_sparsity": pages,
             "block_sparse": blocks,
             "e2e": e2e,

@@ -356,3 +356,27 @@ def test_scoring_shapes(H, Hkv, q, L):
     ref_h, ref_l = oracle.score(x["Q"], x["K"], q)
     assert_scores_close(s_h.cpu().numpy(), ref_h, "s_h")
     assert_scores_close(s_l.cpu().numpy(), ref_l, "s_l")
+
+
+def test_layer_replays_bitwise_in_a_cuda_graph():
+    """The whole layer is stream-capturable: a captured replay equals eager calls."""
+    x = make_inputs(1, 3000, 32, 8, 128, torch.bfloat16, seed=61)
+    d = _dev(x)
+    dm = tsa.dims(d["Q"], d["K"])
+    ws = tsa.workspace(dm, 16, layer=True)
+    Y = torch.empty_like(d["X"])
+    run = lambda: tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=16, tau=0.01, ws=ws)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run()
+    torch.cuda.current_stream().wait_stream(side)
+    want = run().clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    Y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert tsa.tsa_get_device_status(ws) == 0
+    assert torch.equal(Y, want)
