@@ -92,3 +92,26 @@ def test_out_of_range_scores_are_flagged():
     # in-range scores give no error
     tsa.tsa_budget(dm, torch.full((1, 4096), 1.0 / 4096, device="cuda"), 0.01, ws=ws)
     assert tsa.tsa_get_device_status(ws) == 0
+
+
+def test_direct_gather_and_block_modes_time_out_and_recover():
+    """The cp.async producer of the direct-gather mode and the mask walk of the block mode
+    go through the same bounded waits."""
+    d, dm, Lk, Qh, Kh, Vh, s_h, _ = _stage_inputs()
+    idx = tsa.tsa_select(dm, s_h, Lk)
+    ws = tsa.workspace(dm, 16)
+    want_y = tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, d["X"], ws=ws)
+    _, mask = tsa.tsa_block_select(dm, Qh, Kh, Lk, 0.5, logits=False)
+    want_o = tsa.tsa_attn_block(dm, Qh, Kh, Vh, Lk, mask, ws=ws)
+    lk = int(Lk.item())
+    assert tsa.tsa_get_device_status(ws) == 0
+    with stalled():
+        tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, d["X"], ws=ws)
+        st_g = tsa.tsa_get_device_status(ws)
+        tsa.tsa_attn_block(dm, Qh, Kh, Vh, Lk, mask, ws=ws)
+        st_b = tsa.tsa_get_device_status(ws)
+    assert st_g == TIMEOUT and st_b == TIMEOUT
+    assert torch.equal(tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, d["X"], ws=ws), want_y)
+    got_o = tsa.tsa_attn_block(dm, Qh, Kh, Vh, Lk, mask, ws=ws)
+    assert torch.equal(got_o[:, :, :lk], want_o[:, :, :lk])
+    assert tsa.tsa_get_device_status(ws) == 0
