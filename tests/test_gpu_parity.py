@@ -210,8 +210,12 @@ def test_budget_synthetic_scores_bitexact():
     cases.append((v / v.sum()).astype(np.float32))
     cases.append(np.concatenate([np.full(4, 0.25, np.float32), np.zeros(L - 4, np.float32)]))
     cases.append(np.zeros(L, np.float32))                                   # never reached
+    # powers of two from 2^-13 down to subnormals: masses below one unit, exact, shifted
+    w = np.ldexp(np.float32(1.0), -rng.integers(13, 150, size=L)).astype(np.float32)
+    w[::7] *= np.float32(1.75)
+    cases.append(w)
     for s in cases:
-        for tau in (0.0, 0.001, 0.01, 0.25, 0.5, 0.999):
+        for tau in (0.0, 1e-12, 0.001, 0.01, 0.25, 0.5, 0.999):
             dm = tsa.Dims(1, len(s), 1, 1, 64, tsa.TSA_BF16)
             sl = torch.from_numpy(s).cuda().view(1, -1)
             lk = tsa.tsa_budget(dm, sl, tau)
@@ -247,6 +251,35 @@ def test_select_multichunk_ties_bitexact():
         dm = tsa.Dims(B, L, H, 1, 64, tsa.TSA_BF16)
         idx = tsa.tsa_select(dm, torch.from_numpy(s).cuda(), torch.from_numpy(lk).cuda())
         np.testing.assert_array_equal(idx.cpu().numpy(), oracle.select(s, lk), err_msg=str(keeps))
+
+
+@pytest.mark.parametrize("L", [4099, 40001, 70001, 200003, 262144, 262147])
+def test_budget_and_select_every_cluster_size_bitexact(L):
+    """Rows of up to 8 x 32768 scores run budget and selection in one thread-block cluster
+    of 1, 2, 4 or 8 CTAs (here 1, 2, 4, 8, 8); 262147 tokens take the grid-wide kernels.
+    Both equal the oracle bit for bit, with heavy ties, ragged slices and a tied run that
+    crosses the slices."""
+    rng = np.random.default_rng(L)
+    B, H = 2, 3
+    s = (rng.integers(0, 7, size=(B, H, L)) / 8).astype(np.float32)
+    s[1, 2, : L // 2] = np.float32(0.5)
+    s[0, 1] = rng.choice(np.array([0.0, 1e-45, 1e-30, 0.25, 1.0, 3e38], np.float32), size=L)
+    dm = tsa.Dims(B, L, H, 1, 64, tsa.TSA_BF16)
+    s_d = torch.from_numpy(s).cuda()
+    for keeps in ([int(rng.integers(1, L)), L // 2], [1, L - 1], [L, 0]):
+        lk = np.array(keeps, np.int32)
+        idx = tsa.tsa_select(dm, s_d, torch.from_numpy(lk).cuda())
+        np.testing.assert_array_equal(idx.cpu().numpy(), oracle.select(s, lk), err_msg=str(keeps))
+    v = (rng.random((B, L)) ** 4).astype(np.float32)
+    sl = (v / v.sum(1, keepdims=True)).astype(np.float32)
+    sl[1, 1000:3000] = np.float32(1.0 / L)
+    sl_d = torch.from_numpy(sl).cuda()
+    for tau in (0.0, 1e-4, 0.01, 0.3, 0.999):
+        lk = tsa.tsa_budget(dm, sl_d, tau)
+        want, _ = oracle.budget(sl, tau)
+        np.testing.assert_array_equal(lk.cpu().numpy(), want, err_msg=str(tau))
+    zero = torch.zeros(B, L, device="cuda")
+    assert tsa.tsa_budget(dm, zero, 0.01).cpu().tolist() == [0, 0]  # tau never reached
 
 
 def test_dense_attention_gqa_matches_oracle():

@@ -205,6 +205,7 @@ cudaError_t launch_budget(const tsa_dims &dm, const float *s_l, double tau, int3
                           char *ws, cudaStream_t stream) {
     const unsigned long long T = (unsigned long long)ceil(tau * 4611686018427387904.0);
     Control *ctl = reinterpret_cast<Control *>(ws);
+    if (radix_cluster_fits(dm.L)) return launch_budget_cluster(dm, s_l, T, Lkeep, ctl, stream);
     BudgetState *st = reinterpret_cast<BudgetState *>(ws + kBudgetStateOffset);
     char *hist = ws + budget_hist_offset(dm.B);
     cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)dm.B * kBudgetHistBytes, stream);

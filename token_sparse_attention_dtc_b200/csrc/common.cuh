@@ -85,6 +85,14 @@ struct SelectState {
 static_assert(sizeof(SelectState) == 16, "select state is 16 bytes");
 size_t select_end(int B, int H, int L);
 
+// Budget and selection on rows that fit in one thread-block cluster's shared memory
+// (up to 8 x 32768 scores): one launch each.  Longer rows take the grid-wide kernels.
+bool radix_cluster_fits(int L);
+cudaError_t launch_budget_cluster(const tsa_dims &dm, const float *s_l, unsigned long long T,
+                                  int32_t *Lkeep, Control *ctl, cudaStream_t stream);
+cudaError_t launch_select_cluster(const tsa_dims &dm, const float *s_h, const int32_t *Lkeep,
+                                  int32_t *idx, Control *ctl, cudaStream_t stream);
+
 // Host-side count of kernels this library has launched (read by tsa_kernel_launches).
 void note_launches(int n);
 

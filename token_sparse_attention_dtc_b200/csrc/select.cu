@@ -281,6 +281,7 @@ cudaError_t launch_select(const tsa_dims &dm, const float *s_h, const int32_t *L
     const int rows = dm.B * dm.H, nchunks = ceil_div(dm.L, kChunk);
     const SelectLayout y = select_layout(dm.B, dm.H, dm.L);
     Control *ctl = reinterpret_cast<Control *>(ws);
+    if (radix_cluster_fits(dm.L)) return launch_select_cluster(dm, s_h, Lkeep, idx, ctl, stream);
     SelectState *st = reinterpret_cast<SelectState *>(ws + y.states);
     unsigned int *hist = reinterpret_cast<unsigned int *>(ws + y.hist);
     ChunkInfo *ci = reinterpret_cast<ChunkInfo *>(ws + y.chunks);
