@@ -253,15 +253,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ Lkeep, int dense,
           int L, int H, int Hkv, float sl2, __nv_bfloat16 *__restrict__ O, GatherArgs ga,
-          const uint32_t *__restrict__ bmask, Control *ctl, uint64_t limit_ns, int stall) {
+          const uint32_t *__restrict__ bmask, int hgroup, Control *ctl, uint64_t limit_ns,
+          int stall) {
     extern __shared__ uint8_t smem_raw[];
     AttnSmem<D> &sm = *reinterpret_cast<AttnSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int TILE = AttnSmem<D>::TILE, NDB = D / 64;
-    // Head-major order: the CTAs in flight together work on the same head (heaviest pairs
-    // first), so they walk the same K/V tiles at the same pace and share them in L2.
-    const int npairs = ceil_div(L, 2 * kBM);
-    const int bh = blockIdx.x / npairs, pair = npairs - 1 - (int)(blockIdx.x % npairs);
+    // CTA order: groups of `hgroup` heads whose K/V fit in L2 together, one group after
+    // the other; inside a group the heaviest pairs of all its heads come first.  The CTAs in
+    // flight share their heads' K/V tiles in L2, and the light pairs fill the tail.
+    const int npairs = ceil_div(L, 2 * kBM), B_H = gridDim.x / npairs;
+    const int grp = blockIdx.x / (hgroup * npairs), r = blockIdx.x % (hgroup * npairs);
+    const int ghead = min(hgroup, B_H - grp * hgroup);  // heads in this group
+    const int bh = grp * hgroup + r % ghead, pair = npairs - 1 - r / ghead;
     const int b = bh / H, h = bh % H;
     const int Lk = dense ? L : __ldg(Lkeep + b);
     const int i0 = pair * 2 * kBM;  // first row of tile A
@@ -551,9 +555,14 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const long nblocks = (long)ceil_div(dm.L, 2 * kBM) * dm.B * dm.H;
+    // Heads per scheduling group: as many as have K and V (2 * L * D bf16 each, counted
+    // without GQA sharing) within kL2Share bytes.
+    constexpr size_t kL2Share = 64u << 20;
+    const size_t kv_head = (size_t)4 * dm.L * D;
+    const int hgroup = (int)std::max<size_t>(1, std::min<size_t>((size_t)dm.B * dm.H, kL2Share / kv_head));
     k_attn_tc<D, kGather><<<(unsigned)nblocks, kThreads, smem, st>>>(
         tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
-        (__nv_bfloat16 *)O, ga, bmask, ctl, (uint64_t)limit_us * 1000ull, test_stall());
+        (__nv_bfloat16 *)O, ga, bmask, hgroup, ctl, (uint64_t)limit_us * 1000ull, test_stall());
     note_launches(1);
     return cudaGetLastError();
 }
