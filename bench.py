@@ -696,6 +696,49 @@ def run_sweep(args):
         del ws
 
 
+def run_drift(args):
+    """Drift pass (tsa_drift) on Llama-8B-shaped calibration states: 32 layers + 1 states of
+    T tokens x 4096, bf16 and fp32; one JSON line per shape with the HBM roofline.
+
+    Algorithmic bytes: every state read once, (N + 1) * T * d_model * esize; the states are
+    larger than L2 (no flush needed)."""
+    import torch
+
+    from token_sparse_attention_dtc_b200 import tsa
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    pk = _peaks()
+    st = torch.cuda.current_stream(dev)
+    for (N, T, D, dt) in ((32, 4096, 4096, torch.bfloat16), (32, 8192, 4096, torch.bfloat16),
+                          (32, 4096, 4096, torch.float32)):
+        g = torch.Generator(device="cpu").manual_seed(args.seed)
+        h = torch.randn(N + 1, T, D, generator=g).to(dt).to(dev)
+        ws = torch.zeros(tsa.lib().tsa_drift_workspace_size(N, T), dtype=torch.uint8, device=dev)
+        for _ in range(max(args.warmup, 3)):
+            tsa.tsa_drift(h, ws=ws)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        ev[0].record(st)
+        for _ in range(args.steps):
+            tsa.tsa_drift(h, ws=ws)
+        ev[1].record(st)
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / args.steps
+        nbytes = h.numel() * h.element_size()
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        print(json.dumps({
+            "metric": "drift pass ms (tsa_drift: R over N layers and the delta = 0.5 mask)",
+            "value": ms, "unit": "ms", "higher_is_better": False,
+            "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": {"workload": "drift: N=%d layers, T=%d tokens, d_model=%d" % (N, T, D),
+                       "l2": "states %.0f MB, larger than L2; no flush" % (nbytes / 1e6)},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm"], "traffic": None,
+                         "algorithmic_bytes": nbytes}}), flush=True)
+        del h, ws
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -712,6 +755,8 @@ def main():
     ap.add_argument("--stack", action="store_true",
                     help="32-layer stack with the sparse set chosen by the drift pass")
     ap.add_argument("--sweep", action="store_true", help="tau x q sweep, B = 2, L = 64K")
+    ap.add_argument("--drift", action="store_true",
+                    help="drift pass on 32-layer Llama-8B-shaped calibration states")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
@@ -727,6 +772,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args)
+        return
+    if args.drift:
+        run_drift(args)
         return
     if args.impl == "reference":  # rank 0 alone times the oracle; other ranks exit
         run_reference(args, w, L, rank, world)
