@@ -16,7 +16,7 @@ namespace tsa {
 cudaError_t launch_score_simt(const tsa_dims &, const void *, const void *, int, float, float *,
                               const WsLayout &, char *, cudaStream_t);
 cudaError_t launch_score_tc(const tsa_dims &, const void *, const void *, int, float, float *,
-                            const WsLayout &, char *, cudaStream_t, uint32_t);
+                            float *, const WsLayout &, char *, cudaStream_t, uint32_t, bool &);
 cudaError_t launch_fill_lkeep(int, int32_t, int32_t *, cudaStream_t);
 size_t drift_workspace_bytes(int, long long);
 size_t block_scratch_bytes(const tsa_dims &);
@@ -127,13 +127,14 @@ WsLayout ws_layout(const tsa_dims &dm, int q) {
     w.N = (dm.H / dm.Hkv) * w.qe;
     w.nsplit = score_split_cap(dm);
     w.nblk_norm = ceil_div(dm.L, 256);
+    const int norm_slots = std::max(w.nblk_norm, 1024);  // also one per scoring CTA (<= SMs)
     size_t off = align256(sizeof(Control));  // scoring scratch after the control block
     w.score_part = off;
     off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.nsplit * w.N);
     w.score_stat = off;
     off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.N);
     w.norm_part = off;
-    off = align256(off + sizeof(float) * (size_t)dm.B * w.nblk_norm);
+    off = align256(off + sizeof(float) * (size_t)dm.B * norm_slots);
     // the budget and selection scratch overlap the scoring scratch (stages run in order)
     w.total = std::max(off, std::max(budget_end(dm.B), select_end(dm.B, dm.H, dm.L)));
     return w;
@@ -178,11 +179,13 @@ static tsa_status do_score(const tsa_dims &dm, const void *Q, const void *K, int
                            float *s_h, float *s_l, char *ws, cudaStream_t st) {
     const WsLayout w = ws_layout(dm, q);
     cudaError_t e;
+    bool fused = false;  // the tensor-core scoring also wrote s_l
     if (dm.dtype == TSA_BF16)
-        e = launch_score_tc(dm, Q, K, w.qe, scale, s_h, w, ws, st, g_wait_limit_us);
+        e = launch_score_tc(dm, Q, K, w.qe, scale, s_h, s_l, w, ws, st, g_wait_limit_us, fused);
     else
         e = launch_score_simt(dm, Q, K, w.qe, scale, s_h, w, ws, st);
     TSA_TRY(cuda_status(e, "tsa_score"));
+    if (fused) return TSA_OK;
     return cuda_status(launch_norm(dm, s_h, s_l, w, ws, st), "tsa_score (normalise)");
 }
 

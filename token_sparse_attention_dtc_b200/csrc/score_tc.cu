@@ -48,6 +48,8 @@ template <int D> struct ScoreSmem {
     uint64_t stall;     // test hook: initialised, never completed
     alignas(16) float mlog[256];  // pass 2: max + log2(sum) per query row (log2 units)
     float2 red[4][256]; // pass 1: per column group (max, sum) per query row
+    float wsum[16];     // layer score: per epilogue warp partial sums
+    float zsum;         // layer score: the batch element's total
     uint32_t tmem_base;
     int abort, never, gbar_ok;
 };
@@ -91,8 +93,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restrict__ Q, int L,
            int H, int Hkv, int qe, float sl2, int nsplit, int group0, float2 *part,
-           float *__restrict__ s_h, unsigned int *gbar, Control *ctl, uint64_t limit_ns,
-           int stall) {
+           float *__restrict__ s_h, float *__restrict__ s_l, float *__restrict__ norm_part,
+           unsigned int *gbar, Control *ctl, uint64_t limit_ns, int stall) {
     extern __shared__ uint8_t smem_raw[];
     ScoreSmem<D> &sm = *reinterpret_cast<ScoreSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -288,26 +290,36 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                     online_merge(mm, ll, sm.red[g2][n].x, sm.red[g2][n].y);
                 __stcg(&part[((size_t)bg * nsplit + split) * N + n], make_float2(mm, ll));
             }
-        // ---- grid barrier: every CTA's pass-1 pairs are in global memory
-        __threadfence();
-        named_barrier(1, kEpiWarps * 32);
-        if (et == 0) {
-            int good = 0;
-            if (!*abort) {
-                atomicAdd(gbar, 1u);
-                const uint64_t t0 = globaltimer_ns();
-                for (uint32_t k = 0;; ++k) {
-                    unsigned v;
-                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gbar) : "memory");
-                    if (v >= nctas) { good = 1; break; }
-                    if ((k & 63) == 63 && (*abort || globaltimer_ns() - t0 > limit_ns)) break;
-                    __nanosleep(64);
+        // Grid barrier among the epilogue warps of every CTA: the counter (zeroed before the
+        // launch) reaches `target` = nctas times the barrier's ordinal.  Every epilogue
+        // thread must call it (named barriers inside); it returns false when the wait ran
+        // out or the CTA aborted.
+        auto grid_sync = [&](unsigned target) -> bool {
+            __threadfence();
+            named_barrier(1, kEpiWarps * 32);
+            if (et == 0) {
+                int good = 0;
+                if (!*abort) {
+                    atomicAdd(gbar, 1u);
+                    const uint64_t t0 = globaltimer_ns();
+                    for (uint32_t k = 0;; ++k) {
+                        unsigned v;
+                        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gbar) : "memory");
+                        if (v >= target) { good = 1; break; }
+                        if ((k & 63) == 63 && (*abort || globaltimer_ns() - t0 > limit_ns)) break;
+                        __nanosleep(64);
+                    }
                 }
+                sm.gbar_ok = good;
             }
-            sm.gbar_ok = good;
+            named_barrier(1, kEpiWarps * 32);
+            return sm.gbar_ok != 0;
+        };
+        // ---- grid barrier: every CTA's pass-1 pairs are in global memory
+        {
+            const bool g1 = grid_sync(nctas);
+            ok = ok && g1;
         }
-        named_barrier(1, kEpiWarps * 32);
-        ok = ok && sm.gbar_ok;
         // ---- merge the pass-1 pairs of this group in split order: (max, 1/sum) per row
         if (ok && et < N) {
             float mm = -INFINITY, ll = 0.0f;
@@ -363,6 +375,54 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
             tc_fence_before();
             mbar_arrive(&sm.acc_empty[a]);
         }
+        if (s_l) {
+            // ---- layer score in the same launch (it covers every KV group of every batch
+            // element): u[t] = sum_h s_h[h, t] in head order, the per-CTA partial sums, a
+            // grid barrier, then s_l = u / (sum of the partials in CTA order).
+            const bool g2 = grid_sync(2 * nctas);  // every s_h row is written
+            ok = ok && g2;
+            const int cta = blockIdx.y * gridDim.x + blockIdx.x, Bn = gridDim.y / Hkv;
+            const int cl = ceil_div(L, (int)nctas);
+            const int t0 = min(L, cta * cl), t1 = min(L, t0 + cl);
+            const int ew = warp - 4;
+            for (int bb = 0; bb < Bn; ++bb) {
+                float ps = 0.0f;
+                if (ok)
+                    for (int t = t0 + et; t < t1; t += kEpiWarps * 32) {
+                        float u = 0.0f;
+                        for (int h = 0; h < H; ++h) u += __ldcg(s_h + ((size_t)bb * H + h) * L + t);
+                        __stcg(s_l + (size_t)bb * L + t, u);
+                        ps += u;
+                    }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+                if (lane == 0) sm.wsum[ew] = ps;
+                named_barrier(1, kEpiWarps * 32);
+                if (et == 0) {
+                    float z = 0.0f;
+                    for (int w2 = 0; w2 < kEpiWarps; ++w2) z += sm.wsum[w2];
+                    __stcg(norm_part + (size_t)bb * nctas + cta, z);
+                }
+                named_barrier(1, kEpiWarps * 32);  // wsum is free again
+            }
+            const bool g3 = grid_sync(3 * nctas);  // every partial sum is written
+            ok = ok && g3;
+            for (int bb = 0; bb < Bn; ++bb) {
+                if (ew == 0) {
+                    float z = 0.0f;
+                    for (int c = lane; c < (int)nctas; c += 32) z += __ldcg(norm_part + (size_t)bb * nctas + c);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                    if (lane == 0) sm.zsum = z;
+                }
+                named_barrier(1, kEpiWarps * 32);
+                const float Z = sm.zsum;
+                if (ok)
+                    for (int t = t0 + et; t < t1; t += kEpiWarps * 32)
+                        s_l[(size_t)bb * L + t] = __ldcg(s_l + (size_t)bb * L + t) / Z;
+                named_barrier(1, kEpiWarps * 32);  // zsum is free again
+            }
+        }
     }
     if (!ok) {
         *abort = 1;
@@ -400,8 +460,8 @@ int score_tc_splits(const tsa_dims &dm) {
 
 template <int D>
 static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *K, int qe,
-                                 float scale, float *s_h, const WsLayout &w, char *ws,
-                                 cudaStream_t st, uint32_t limit_us) {
+                                 float scale, float *s_h, float *s_l, const WsLayout &w, char *ws,
+                                 cudaStream_t st, uint32_t limit_us, bool &fused) {
     CUtensorMap tk;
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)dm.L, (uint64_t)dm.Hkv, (uint64_t)dm.B};
     const uint64_t strides[3] = {(uint64_t)dm.Hkv * D * 2, (uint64_t)D * 2,
@@ -424,12 +484,17 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
     const __nv_bfloat16 *Qb = (const __nv_bfloat16 *)Q;
     int L = dm.L, H = dm.H, Hkv = dm.Hkv;
     const int groups = dm.B * dm.Hkv, per_launch = std::min(groups, sm_count());
+    // One launch covering every group also computes the layer score.
+    fused = per_launch == groups && s_l != nullptr;
+    float *sl = fused ? s_l : nullptr;
+    float *np = reinterpret_cast<float *>(ws + w.norm_part);
     for (int g0 = 0; g0 < groups; g0 += per_launch) {
         int group0 = g0;
         const int gc = std::min(per_launch, groups - g0);
         if ((e = cudaMemsetAsync(gbar, 0, sizeof(unsigned int), st))) return e;
         void *args[] = {&tk, (void *)&Qb, &L, &H, &Hkv, &qe, &sl2, &nsplit, &group0,
-                        (void *)&part, (void *)&s_h, (void *)&gbar, (void *)&ctl, &lim, &stall};
+                        (void *)&part, (void *)&s_h, (void *)&sl, (void *)&np, (void *)&gbar,
+                        (void *)&ctl, &lim, &stall};
         e = cudaLaunchCooperativeKernel((const void *)k_score_tc<D>, dim3(nsplit, gc),
                                         dim3(kThreads), args, smem, st);
         if (e != cudaSuccess) return e;
@@ -438,11 +503,13 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
     return cudaSuccess;
 }
 
+// s_l may be NULL (no layer score); `fused` tells the caller whether s_l was written.
 cudaError_t launch_score_tc(const tsa_dims &dm, const void *Q, const void *K, int qe,
-                            float scale, float *s_h, const WsLayout &w, char *ws,
-                            cudaStream_t st, uint32_t limit_us) {
-    return dm.d == 64 ? score_tc_impl<64>(dm, Q, K, qe, scale, s_h, w, ws, st, limit_us)
-                      : score_tc_impl<128>(dm, Q, K, qe, scale, s_h, w, ws, st, limit_us);
+                            float scale, float *s_h, float *s_l, const WsLayout &w, char *ws,
+                            cudaStream_t st, uint32_t limit_us, bool &fused) {
+    return dm.d == 64
+               ? score_tc_impl<64>(dm, Q, K, qe, scale, s_h, s_l, w, ws, st, limit_us, fused)
+               : score_tc_impl<128>(dm, Q, K, qe, scale, s_h, s_l, w, ws, st, limit_us, fused);
 }
 
 }  // namespace tsa
