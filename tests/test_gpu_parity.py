@@ -391,6 +391,20 @@ def test_scoring_shapes(H, Hkv, q, L):
     assert_scores_close(s_l.cpu().numpy(), ref_l, "s_l")
 
 
+def test_scoring_many_groups_takes_several_launches():
+    """B * Hkv = 160 KV groups exceed one cooperative launch (one CTA per SM): the scoring
+    runs in two launches and the layer score in its own kernels.  Both paths equal the
+    oracle; a 2-sample batch (one launch, layer score inside the scoring kernel) checks
+    the fused path with B > 1."""
+    for B, Hkv, L in ((20, 8, 200), (2, 8, 700)):
+        x = make_inputs(B, L, Hkv * 2, Hkv, 64, torch.bfloat16, seed=B)
+        d = _dev(x)
+        s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16)
+        ref_h, ref_l = oracle.score(x["Q"], x["K"], 16)
+        assert_scores_close(s_h.cpu().numpy(), ref_h, "s_h B=%d" % B)
+        assert_scores_close(s_l.cpu().numpy(), ref_l, "s_l B=%d" % B)
+
+
 def test_layer_replays_bitwise_in_a_cuda_graph():
     """The whole layer is stream-capturable: a captured replay equals eager calls."""
     x = make_inputs(1, 3000, 32, 8, 128, torch.bfloat16, seed=61)

@@ -14,9 +14,10 @@
 // fp32 (lanes, then a fixed butterfly), the ratio is accumulated in fp64 in the warp's own
 // shared-memory row, and the blocks' partials are summed in a fixed order, so R does not
 // depend on scheduling.
-#include "common.cuh"
+#include "sm100.cuh"
 
 namespace tsa {
+using namespace sm100;
 
 namespace {
 
@@ -25,27 +26,32 @@ namespace {
 constexpr int kDriftWarps = 8, kDriftTokensPerWarp = 1;
 constexpr int kDriftTokensPerBlock = kDriftWarps * kDriftTokensPerWarp;
 
-__device__ inline void acc_pair(const uint4 &a, const uint4 &b, float &dd, float &hh, float) {
+// Adds |b - a|^2 and |a|^2 of one 16-byte vector into the pairs (dd[0], dd[1]) and
+// (hh[0], hh[1]) (even and odd elements), with paired fp32 instructions.
+__device__ inline void acc_pair(const uint4 &a, const uint4 &b, float (&dd)[2], float (&hh)[2],
+                                float) {
     const float *x = reinterpret_cast<const float *>(&a), *y = reinterpret_cast<const float *>(&b);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float d = y[i] - x[i];
-        dd = fmaf(d, d, dd);
-        hh = fmaf(x[i], x[i], hh);
+    for (int i = 0; i < 4; i += 2) {
+        float d0, d1;
+        sub2(d0, d1, y[i], y[i + 1], x[i], x[i + 1]);
+        fma2(dd[0], dd[1], d0, d1, d0, d1, dd[0], dd[1]);
+        fma2(hh[0], hh[1], x[i], x[i + 1], x[i], x[i + 1], hh[0], hh[1]);
     }
 }
-__device__ inline void acc_pair(const uint4 &a, const uint4 &b, float &dd, float &hh,
+// bf16: the low element of a word is its low 16 bits shifted up, the high one its high 16
+// bits masked (exact conversions).
+__device__ inline void acc_pair(const uint4 &a, const uint4 &b, float (&dd)[2], float (&hh)[2],
                                 __nv_bfloat16) {
-    const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
-    const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
+    const uint32_t xa[4] = {a.x, a.y, a.z, a.w}, yb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float2 xf = __bfloat1622float2(x[i]), yf = __bfloat1622float2(y[i]);
-        const float d0 = yf.x - xf.x, d1 = yf.y - xf.y;
-        dd = fmaf(d0, d0, dd);
-        dd = fmaf(d1, d1, dd);
-        hh = fmaf(xf.x, xf.x, hh);
-        hh = fmaf(xf.y, xf.y, hh);
+        const float x0 = __uint_as_float(xa[i] << 16), x1 = __uint_as_float(xa[i] & 0xffff0000u);
+        const float y0 = __uint_as_float(yb[i] << 16), y1 = __uint_as_float(yb[i] & 0xffff0000u);
+        float d0, d1;
+        sub2(d0, d1, y0, y1, x0, x1);
+        fma2(dd[0], dd[1], d0, d1, d0, d1, dd[0], dd[1]);
+        fma2(hh[0], hh[1], x0, x1, x0, x1, hh[0], hh[1]);
     }
 }
 
@@ -65,9 +71,10 @@ k_drift_partial(const uint4 *__restrict__ h, int N, long long Ttok, int vec_per_
         for (int l = 0; l < N; ++l) {
             const uint4 *a = h + (size_t)l * state + (size_t)t * vec_per_row;
             const uint4 *b = a + state;
-            float dd = 0.0f, hh = 0.0f;
+            float d2[2] = {0.0f, 0.0f}, h2[2] = {0.0f, 0.0f};
 #pragma unroll 4
-            for (int v = lane; v < vec_per_row; v += 32) acc_pair(a[v], b[v], dd, hh, T());
+            for (int v = lane; v < vec_per_row; v += 32) acc_pair(a[v], b[v], d2, h2, T());
+            float dd = d2[0] + d2[1], hh = h2[0] + h2[1];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 dd += __shfl_xor_sync(0xffffffffu, dd, o);
@@ -106,9 +113,10 @@ k_drift_partial_reg(const uint4 *__restrict__ h, int N, long long Ttok, float ep
             uint4 nxt[V];
 #pragma unroll
             for (int v = 0; v < V; ++v) nxt[v] = __ldcs(row + v * 32);
-            float dd = 0.0f, hh = 0.0f;
+            float d2[2] = {0.0f, 0.0f}, h2[2] = {0.0f, 0.0f};
 #pragma unroll
-            for (int v = 0; v < V; ++v) acc_pair(cur[v], nxt[v], dd, hh, T());
+            for (int v = 0; v < V; ++v) acc_pair(cur[v], nxt[v], d2, h2, T());
+            float dd = d2[0] + d2[1], hh = h2[0] + h2[1];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 dd += __shfl_xor_sync(0xffffffffu, dd, o);
