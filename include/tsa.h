@@ -57,7 +57,7 @@ typedef enum {
     TSA_OK = 0,
     TSA_ERR_INVALID_ARG = 1,    /* a null pointer, a bad size, tau or scale      */
     TSA_ERR_ALIGNMENT = 2,      /* a pointer that is not 16-byte aligned          */
-    TSA_ERR_UNSUPPORTED = 3,    /* a shape or dtype this build does not implement */
+    TSA_ERR_UNSUPPORTED = 3,    /* a shape or dtype the library does not implement */
     TSA_ERR_WORKSPACE = 4,      /* workspace too small or misaligned              */
     TSA_ERR_CUDA = 5,           /* a CUDA runtime or launch error                 */
     TSA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait ran out             */
