@@ -171,9 +171,10 @@ def _staged(d, dm, Lk, idx):
     return tsa.tsa_scatter_residual(dm, Oh, idx, Lk, d["X"])
 
 
-@pytest.mark.parametrize("B,L,H,Hkv", [(1, 4096, 32, 8), (2, 1000, 8, 2), (2, 5000, 8, 8)])
-def test_attn_gather_equals_staged_path_bitwise(B, L, H, Hkv):
-    x = make_inputs(B, L, H, Hkv, 128, torch.bfloat16, seed=L + H)
+@pytest.mark.parametrize("B,L,H,Hkv,hd", [(1, 4096, 32, 8, 128), (2, 1000, 8, 2, 128),
+                                           (2, 5000, 8, 8, 128), (2, 1500, 8, 2, 64)])
+def test_attn_gather_equals_staged_path_bitwise(B, L, H, Hkv, hd):
+    x = make_inputs(B, L, H, Hkv, hd, torch.bfloat16, seed=L + H)
     d = {k: v.cuda() for k, v in x.items()}
     dm = tsa.dims(d["Q"], d["K"])
     s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16)

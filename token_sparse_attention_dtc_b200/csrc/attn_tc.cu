@@ -38,6 +38,8 @@ using namespace sm100;
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kStages = 2, kThreads = 320;
+// Direct-gather mode: warps 10 and 11 join warp 0 as copy producers (384 threads).
+constexpr int kGatherWarps = 3, kGatherThreads = kThreads + 64;
 constexpr uint64_t kDrainNs = 1000000000ull;  // drain waits: 1 s
 
 template <int D> struct AttnSmem {
@@ -48,7 +50,7 @@ template <int D> struct AttnSmem {
     uint64_t q_full, k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
     uint64_t s_full[2], p_full[2], o_final[2], drain;
     uint64_t stall;  // test hook: initialised, never completed
-    int32_t gidx[2][kBM];  // direct-gather mode: token indices of the tiles being copied
+    int64_t goff[kGatherWarps][2][kBM];  // direct-gather mode: each producer's row offsets
     uint32_t tmem_base;
     int abort;
     int never;  // stays 0: drain waits ignore the abort flag
@@ -63,28 +65,33 @@ struct GatherArgs {
     __nv_bfloat16 *Y;                // [B, L, H*d], may be X
 };
 
-// Producer of the direct-gather mode (all 32 lanes of warp 0).  A 128-row tile of
-// positions p0..p0+127 is copied with 16-byte cp.async into the 128-byte-swizzle layout
-// the MMA descriptors read (16-byte chunk k of row r at r*128 + ((k ^ (r & 7)) * 16) in
-// each 64-column block), row p taken from token idx[p] (p clamped to L - 1; rows past L'
-// are masked or never stored).  One commit group per tile; once the group before the
-// newest has landed, each lane fences (generic -> async proxy) and arrives on its full
-// barrier (32 arrivals).
+// Producer of the direct-gather mode: producer warp pw (0..kGatherWarps-1, all 32 lanes)
+// copies its share of every tile.  A 128-row tile of positions p0..p0+127 is copied with
+// 16-byte cp.async into the 128-byte-swizzle layout the MMA descriptors read (16-byte
+// chunk k of row r at r*128 + ((k ^ (r & 7)) * 16) in each 64-column block), row p taken
+// from token idx[p] (p clamped to L - 1; rows past L' are masked or never stored); warp pw
+// takes the row groups pw, pw + kGatherWarps, ... of 32/CPR rows.  After issuing its share
+// of a tile each lane hands its arrival on the tile's full barrier to the copy engine
+// (cp.async.mbarrier.arrive: the arrival lands with the lane's copies; 32 per producer
+// warp), so no producer waits for its own copies; the MMA thread fences generic -> async
+// proxy after the barrier completes.
 template <int D>
-__device__ __forceinline__ bool gather_producer(AttnSmem<D> &sm, const GatherArgs &ga, int b,
-                                                int h, int kvh, int L, int H, int Hkv, int i0,
-                                                bool hasB, int nkv, int lane, Control *ctl,
+__device__ __forceinline__ bool gather_producer(AttnSmem<D> &sm, const GatherArgs &ga, int pw,
+                                                int b, int h, int kvh, int L, int H, int Hkv,
+                                                int i0, bool hasB, int nkv, int lane, Control *ctl,
                                                 uint64_t limit_ns, volatile int *abort) {
     constexpr int CPR = D / 8;  // 16-byte chunks per row
     const int32_t *S = ga.idx + ((size_t)b * H + h) * L;
     bool bad = false;
     // Token indices of rows p0 + 4*lane .. p0 + 4*lane + 3 (clamped to L - 1), loaded in
-    // one round trip; staged in shared memory so the copy loop has no global dependence.
+    // one round trip; staged in shared memory as element offsets of the rows
+    // ((b * L + t) * heads + head) * D, so the copy loop has no global dependence and no
+    // index arithmetic (K and V share the offsets of a step).
     auto load_idx = [&](int p0, int (&v)[4]) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) v[e] = __ldg(S + min(p0 + 4 * lane + e, L - 1));
     };
-    auto stage_idx = [&](int slot, const int (&v)[4]) {
+    auto stage_idx = [&](int slot, const int (&v)[4], int heads, int head) {
         __syncwarp();  // the previous copy loop has read this slot
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -93,64 +100,50 @@ __device__ __forceinline__ bool gather_producer(AttnSmem<D> &sm, const GatherArg
                 bad = true;
                 t = 0;
             }
-            sm.gidx[slot][4 * lane + e] = t;
+            sm.goff[pw][slot][4 * lane + e] = (((int64_t)b * L + t) * heads + head) * D;
         }
         __syncwarp();
     };
-    auto tile = [&](uint8_t *dst, const __nv_bfloat16 *src, int heads, int head, int slot) {
+    auto tile = [&](uint8_t *dst, const __nv_bfloat16 *src, int slot) {
         const uint32_t d0 = smem_u32(dst);
         const int c = lane % CPR;
         const uint32_t coff = (uint32_t)(c / 8) * (kBM * 128);
-        const __nv_bfloat16 *base = src + (size_t)head * D + c * 8;
-#pragma unroll 8
-        for (int r = lane / CPR; r < kBM; r += 32 / CPR) {
-            const int t = sm.gidx[slot][r];
-            cp_async16(d0 + coff + r * 128 + (((c % 8) ^ (r & 7)) << 4),
-                       base + ((size_t)b * L + t) * heads * D);
-        }
+        const __nv_bfloat16 *base = src + c * 8;
+        constexpr int RPI = 32 / CPR;  // rows per warp iteration
+#pragma unroll 4
+        for (int r = pw * RPI + lane / CPR; r < kBM; r += kGatherWarps * RPI)
+            cp_async16(d0 + coff + r * 128 + (((c % 8) ^ (r & 7)) << 4), base + sm.goff[pw][slot][r]);
     };
-    uint64_t *pending = nullptr;
-    auto publish_previous = [&]() {
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        if (pending) mbar_arrive(pending);
-    };
+
     int va[4], vb[4];
     load_idx(i0, va);
     if (hasB) load_idx(i0 + kBM, vb);
-    stage_idx(0, va);
-    tile(sm.q[0], ga.Q, H, h, 0);
+    stage_idx(0, va, H, h);
+    tile(sm.q[0], ga.Q, 0);
     if (hasB) {
-        stage_idx(1, vb);
-        tile(sm.q[1], ga.Q, H, h, 1);
+        stage_idx(1, vb, H, h);
+        tile(sm.q[1], ga.Q, 1);
     }
-    cp_async_commit();
-    pending = &sm.q_full;
+    cp_async_mbar_arrive(&sm.q_full);
     int nxt[4];
     if (nkv > 0) load_idx(0, nxt);
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
         const int s = j % kStages, slot = j & 1;
         const uint32_t ph = ((j / kStages) & 1) ^ 1;
-        stage_idx(slot, nxt);
+        stage_idx(slot, nxt, Hkv, kvh);
         if (j + 1 < nkv) load_idx((j + 1) * kBN, nxt);  // in flight during this step's copies
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.k_empty[s], ph, limit_ns, abort));
         if (!ok) break;
-        tile(sm.k[s], ga.K, Hkv, kvh, slot);
-        cp_async_commit();
-        publish_previous();
-        pending = &sm.k_full[s];
+        tile(sm.k[s], ga.K, slot);
+        cp_async_mbar_arrive(&sm.k_full[s]);
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[s], ph, limit_ns, abort));
         if (!ok) break;
-        tile(sm.v[s], ga.V, Hkv, kvh, slot);
-        cp_async_commit();
-        publish_previous();
-        pending = &sm.v_full[s];
+        tile(sm.v[s], ga.V, slot);
+        cp_async_mbar_arrive(&sm.v_full[s]);
     }
-    // Drain: every copy of this lane lands before the CTA can exit; publish the last tile.
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (ok) mbar_arrive(pending);
+    // Drain: every copy of this lane lands before the CTA can exit.
+    cp_async_wait_all();
     if (__any_sync(0xffffffffu, bad) && lane == 0) report_error(ctl, TSA_ERR_INVALID_ARG, 31);
     return ok;
 }
@@ -249,7 +242,7 @@ __device__ __forceinline__ bool softmax_tile(AttnSmem<D> &sm, int X, int n, uint
 }
 
 template <int D, bool kGather>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGather ? kGatherThreads : kThreads, 1)
 k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
           const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ Lkeep, int dense,
           int L, int H, int Hkv, float sl2, __nv_bfloat16 *__restrict__ O, GatherArgs ga,
@@ -292,7 +285,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        const uint32_t nfill = kGather ? 32 : 1;  // cp.async lanes, or one TMA thread
+        const uint32_t nfill = kGather ? 32 * kGatherWarps : 1;  // cp.async lanes, or one TMA thread
         mbar_init(&sm.q_full, nfill);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.k_full[s], nfill);
@@ -321,9 +314,9 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const uint32_t tmem = sm.tmem_base;
     volatile int *abort = &sm.abort;
     bool ok = true;
-    if (warp == 0 && kGather) {
-        ok = gather_producer<D>(sm, ga, b, h, kvh, L, H, Hkv, i0, hasB, nkv, lane, ctl, limit_ns,
-                                abort);
+    if (kGather && (warp == 0 || warp >= 10)) {
+        ok = gather_producer<D>(sm, ga, warp == 0 ? 0 : warp - 9, b, h, kvh, L, H, Hkv, i0, hasB,
+                                nkv, lane, ctl, limit_ns, abort);
     } else if (warp == 0) {
         if (lane == 0) {
             int issued = 0;  // K/V tiles issued (negative: K of tile -issued-1 only)
@@ -401,6 +394,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             ok = ok && mbar_wait(&sm.q_full, 0, limit_ns, abort) &&
                  mbar_wait(&sm.k_full[0], 0, limit_ns, abort);
             if (ok) {
+                if (kGather) fence_proxy_async_smem();  // cp.async writes -> the MMA's reads
                 tc_fence_after();
                 S_mma(0, 0);
                 if (hasB) S_mma(1, 0);
@@ -413,6 +407,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 if (next && !(ok = mbar_wait(&sm.k_full[(j + 1) % kStages],
                                              ((j + 1) / kStages) & 1, limit_ns, abort)))
                     break;
+                if (kGather) fence_proxy_async_smem();  // cp.async writes -> the MMA's reads
                 for (int x = 0; x < 2; ++x) {
                     const int nx = x ? nB : nA;
                     if (j >= nx) continue;
@@ -560,7 +555,7 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
     constexpr size_t kL2Share = 64u << 20;
     const size_t kv_head = (size_t)4 * dm.L * D;
     const int hgroup = (int)std::max<size_t>(1, std::min<size_t>((size_t)dm.B * dm.H, kL2Share / kv_head));
-    k_attn_tc<D, kGather><<<(unsigned)nblocks, kThreads, smem, st>>>(
+    k_attn_tc<D, kGather><<<(unsigned)nblocks, kGather ? kGatherThreads : kThreads, smem, st>>>(
         tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
         (__nv_bfloat16 *)O, ga, bmask, hgroup, ctl, (uint64_t)limit_us * 1000ull, test_stall());
     note_launches(1);
