@@ -521,3 +521,23 @@ def test_block_attention_matches_masked_softmax():
         rows = [(0, h, i) for i in range(0, 640, 7)]
         got = oracle.attend_block_rows(x["Q"], x["K"], x["V"], idx, lk, keep, rows)
         np.testing.assert_allclose(got, ref[::7].numpy(), rtol=0, atol=1e-13)
+
+
+def test_oracle_matches_its_stored_regression():
+    """The oracle reproduces, bit for bit, the results it stored for one small seeded layer
+    (tests/golden/make_oracle_regression.py).  This pins the oracle against unintended
+    changes of its arithmetic; the pins above pin it against the pages and mathematics."""
+    import importlib.util
+    import json
+    import os
+
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location(
+        "make_oracle_regression", os.path.join(here, "make_oracle_regression.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    with open(os.path.join(here, "oracle_regression.json")) as f:
+        want = json.load(f)
+    got = json.loads(json.dumps(mod.compute()))
+    for k in ("case", "Lkeep", "idx", "s_l", "s_h", "Oh", "Y"):
+        assert got[k] == want[k], k
