@@ -153,6 +153,16 @@ def test_recent_queries_exceed_length():
     check_layer(x, 16, 0.05, g)
 
 
+@pytest.mark.parametrize("L", [1, 2, 129])
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_shortest_sequences(L, dtype, d):
+    """One token (the budget then prunes it: L' = 0, Y = X), two tokens, and one token past
+    a full 128-row tile, with two samples."""
+    x = make_inputs(2, L, 4, 2, d, dtype, seed=L)
+    g = run_stages(x, 16, 0.05)
+    check_layer(x, 16, 0.05, g)
+
+
 def test_tau_zero_keeps_everything_and_matches_dense():
     x = make_inputs(1, 300, 4, 1, 128, torch.bfloat16, seed=5)
     g = run_stages(x, 16, 0.0)
