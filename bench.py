@@ -578,13 +578,15 @@ def run_stack(args, L):
     ws = tsa.workspace(dm, q, layer=True, device=dev)
     X = X0.clone()
     st = torch.cuda.current_stream(dev)
+    # L' of each sparse layer: rows of 4 int32, since optional outputs are 16-byte aligned
+    Lk = torch.zeros(n_layers, 4, dtype=torch.int32, device=dev)
 
     def stack(mask):
         X.copy_(X0)
         for l in range(n_layers):
             c = layers[l]
             tsa.tsa_layer(c["Q"], c["K"], c["V"], X, X, is_sparse=bool(mask[l]), q=q, tau=tau,
-                          ws=ws)
+                          Lkeep=Lk[l, :1], ws=ws)
 
     # calibration: all dense, keep every state for the drift pass
     states = torch.empty(n_layers + 1, L, H * dd, dtype=torch.bfloat16, device=dev)
@@ -645,6 +647,7 @@ def run_stack(args, L):
         "eager_ms": eager_ms, "graph": graph, "all_dense_ms": dense_ms,
         "speedup_vs_all_dense": dense_ms / (graph["replay_ms"] or eager_ms),
         "sparse_layers": [l for l in range(n_layers) if mask[l]],
+        "sparse_kept": [int(Lk[l, 0]) for l in range(n_layers) if mask[l]],
         "drift_R": [round(float(v), 6) for v in R.cpu()],
         "gpu_launches_per_stack": launches,
     }
