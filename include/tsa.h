@@ -324,6 +324,20 @@ TSA_API void tsa_set_wait_limit(uint32_t microseconds);
  * down as described above, and exits.  Nothing faults, traps or hangs. */
 TSA_API void tsa_set_test_stall(int32_t on);
 
+/* Scoring schedule of bf16 inputs, for tests and measurements; default (0, 0).  With
+ * wave = 0 every bf16 shape takes the single-wave kernel: every KV group at once, K read
+ * from HBM twice (once per softmax pass).  With wave = 1, shapes of 16 recent queries
+ * (q >= 16 and L >= 16) and at most 4 query heads per KV head take the wave-scheduled
+ * kernel instead: the KV groups a few at a time (about 40 MB of K per wave), so that the
+ * second pass rereads K from L2 and K crosses HBM once.  The single-wave kernel is the
+ * default because it is as fast or faster on one B200 at every length measured (the
+ * wave schedule's tile pipeline is no faster from L2 than from HBM, and its passes run
+ * one after the other).  max_groups_per_wave > 0 caps the groups of one wave (more
+ * waves on small inputs); 0 lets the library choose.  Both kernels give the scores
+ * tsa_score defines, within fp32 rounding; they differ in summation order only.
+ * Applies to later launches from any thread. */
+TSA_API void tsa_set_score_schedule(int32_t wave, int32_t max_groups_per_wave);
+
 /* Number of CUDA kernels this library has launched in this process, on every device and
  * thread (a host-side counter; memset and copy operations are not counted).  Callers take
  * the difference around a region to count its launches.  Never fails. */

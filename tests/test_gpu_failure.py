@@ -64,16 +64,27 @@ def test_attention_wait_timeout_is_reported_and_context_recovers():
     assert st == TIMEOUT
 
 
-def test_scoring_wait_timeout_is_reported_and_context_recovers():
+@pytest.mark.parametrize("wave", [True, False])
+def test_scoring_wait_timeout_is_reported_and_context_recovers(wave):
+    """Both scoring kernels (the single-wave default and the wave-scheduled one, which
+    this shape takes when asked) time out, report it, and score correctly afterwards."""
     d, dm, _, _, _, _, s_h_ref, s_l_ref = _stage_inputs()
     ws = tsa.workspace(dm, 16)
-    with stalled():
-        tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
-        st = tsa.tsa_get_device_status(ws)
-    assert st == TIMEOUT
-    s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
-    assert tsa.tsa_get_device_status(ws) == 0
-    assert torch.equal(s_h, s_h_ref) and torch.equal(s_l, s_l_ref)
+    tsa.tsa_set_score_schedule(wave, 0)
+    try:
+        with stalled():
+            tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
+            st = tsa.tsa_get_device_status(ws)
+        assert st == TIMEOUT
+        s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16, ws=ws)
+        assert tsa.tsa_get_device_status(ws) == 0
+    finally:
+        tsa.tsa_set_score_schedule(False, 0)
+    if not wave:
+        assert torch.equal(s_h, s_h_ref) and torch.equal(s_l, s_l_ref)
+    else:  # the reference scores came from the default (single-wave) kernel
+        torch.testing.assert_close(s_h, s_h_ref, rtol=1e-5, atol=1e-30)
+        torch.testing.assert_close(s_l, s_l_ref, rtol=1e-5, atol=1e-30)
 
 
 def test_out_of_range_scores_are_flagged():

@@ -402,10 +402,12 @@ def test_scoring_shapes(H, Hkv, q, L):
 
 
 def test_scoring_many_groups_takes_several_launches():
-    """B * Hkv = 160 KV groups exceed one cooperative launch (one CTA per SM): the scoring
-    runs in two launches and the layer score in its own kernels.  Both paths equal the
-    oracle; a 2-sample batch (one launch, layer score inside the scoring kernel) checks
-    the fused path with B > 1."""
+    """Single-wave kernel (the default): B * Hkv = 160 KV groups exceed one cooperative
+    launch (one CTA per SM), so the scoring runs in two launches and the layer score in
+    its own kernels.  Both paths equal the oracle; a 2-sample batch (one launch, layer
+    score inside the scoring kernel) checks the fused path with B > 1.  (The opt-in
+    wave-scheduled kernel covers any number of groups in one launch; its tests are in
+    test_gpu_score_wave.py.)"""
     for B, Hkv, L in ((20, 8, 200), (2, 8, 700)):
         x = make_inputs(B, L, Hkv * 2, Hkv, 64, torch.bfloat16, seed=B)
         d = _dev(x)

@@ -51,8 +51,11 @@ cudaError_t launch_scatter(const tsa_dims &, const void *, const int32_t *, cons
 static thread_local std::string g_last_error;
 static uint32_t g_wait_limit_us = 2000000;  // 2 s
 static int g_test_stall = 0;
+static int g_score_wave = 0, g_score_wave_cap = 0;
 
 int test_stall() { return g_test_stall; }
+bool force_single_wave() { return g_score_wave == 0; }  // the default
+int score_wave_group_cap() { return g_score_wave_cap; }
 
 static std::atomic<uint64_t> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -127,10 +130,13 @@ WsLayout ws_layout(const tsa_dims &dm, int q) {
     w.N = (dm.H / dm.Hkv) * w.qe;
     w.nsplit = score_split_cap(dm);
     w.nblk_norm = ceil_div(dm.L, 256);
-    const int norm_slots = std::max(w.nblk_norm, 1024);  // also one per scoring CTA (<= SMs)
+    // also 16 warp totals per scoring CTA (<= 160 CTAs) of the fused layer score
+    const int norm_slots = std::max(w.nblk_norm, 160 * 16);
     size_t off = align256(sizeof(Control));  // scoring scratch after the control block
+    const bool wave = dm.dtype == TSA_BF16;  // room for the wave-scheduled scoring too
     w.score_part = off;
-    off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.nsplit * w.N);
+    off = align256(off + std::max(sizeof(float2) * (size_t)dm.B * dm.Hkv * w.nsplit * w.N,
+                                  wave ? score_wave_bytes(dm.B) : size_t(0)));
     w.score_stat = off;
     off = align256(off + sizeof(float2) * (size_t)dm.B * dm.Hkv * w.N);
     w.norm_part = off;
@@ -586,6 +592,11 @@ tsa_status tsa_get_device_status(void *ws, void *stream) {
 void tsa_set_wait_limit(uint32_t microseconds) { g_wait_limit_us = microseconds; }
 
 void tsa_set_test_stall(int32_t on) { g_test_stall = on ? 1 : 0; }
+
+void tsa_set_score_schedule(int32_t wave, int32_t max_groups_per_wave) {
+    g_score_wave = wave ? 1 : 0;
+    g_score_wave_cap = max_groups_per_wave > 0 ? max_groups_per_wave : 0;
+}
 
 uint64_t tsa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 

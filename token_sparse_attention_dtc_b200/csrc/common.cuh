@@ -18,6 +18,11 @@ struct Control {
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
 constexpr int kScoreSplitTokens = 4096;  // tokens per scoring split (SIMT path)
+// Scratch of the wave-scheduled tensor-core scoring: float2 per-CTA (max, sum) pairs of
+// 4 wave slots x up to 160 CTAs x 64 query rows, then float per-warp layer-score totals
+// [B][up to 160 CTAs][16 warps].
+constexpr size_t kScoreWavePartBytes = size_t(4) * 160 * 64 * 8;
+inline size_t score_wave_bytes(int B) { return kScoreWavePartBytes + size_t(B) * 160 * 16 * 4; }
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -124,5 +129,10 @@ inline int score_split_cap(const tsa_dims &dm) {
 
 // Host: the failure-path test hook set by tsa_set_test_stall (0 or 1).
 int test_stall();
+// Host: true (the default) unless tsa_set_score_schedule(1, ...) lets the shapes it
+// covers take the wave-scheduled scoring kernel.
+bool force_single_wave();
+// Host: the cap on KV groups per wave set by tsa_set_score_schedule (0: none).
+int score_wave_group_cap();
 
 }  // namespace tsa

@@ -34,6 +34,12 @@
 namespace tsa {
 using namespace sm100;
 
+// The wave-scheduled kernel (score_wave.cu) takes the shapes it covers.
+bool score_wave_eligible(const tsa_dims &dm, int qe);
+cudaError_t launch_score_wave(const tsa_dims &dm, const void *Q, const void *K, float scale,
+                              float *s_h, float *s_l, const WsLayout &w, char *ws,
+                              cudaStream_t st, uint32_t limit_us);
+
 namespace {
 
 constexpr int kThreads = 640, kStages = 4, kTile = 128;
@@ -49,7 +55,6 @@ template <int D> struct ScoreSmem {
     alignas(16) float mlog[256];  // pass 2: max + log2(sum) per query row (log2 units)
     float2 red[4][256]; // pass 1: per column group (max, sum) per query row
     float wsum[16];     // layer score: per epilogue warp partial sums
-    float zsum;         // layer score: the batch element's total
     uint32_t tmem_base;
     int abort, never, gbar_ok;
 };
@@ -332,6 +337,8 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
         named_barrier(1, kEpiWarps * 32);
         // ---- pass 2: thread owns token r of the tile and the heads g = cg, cg + 4, ...;
         // head g's query rows are the columns [g*qe, (g+1)*qe), summed in row order.
+        // zs: this thread's sum of the s_h values it writes (for the layer score's total).
+        float zs = 0.0f;
         for (int it = count; it < total && ok; ++it) {
             const int a = it & (nbuf - 1);
             ok = mbar_wait(&sm.acc_full[a], (it >> lgb) & 1, limit_ns, abort);
@@ -370,57 +377,57 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                     }
                 }
                 acc += a0 + a1;
-                if (t < L) s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
+                if (t < L) {
+                    s_h[((size_t)b * H + kv * G + g) * L + t] = acc;
+                    zs += acc;
+                }
             }
             tc_fence_before();
             mbar_arrive(&sm.acc_empty[a]);
         }
         if (s_l) {
             // ---- layer score in the same launch (it covers every KV group of every batch
-            // element): u[t] = sum_h s_h[h, t] in head order, the per-CTA partial sums, a
-            // grid barrier, then s_l = u / (sum of the partials in CTA order).
-            const bool g2 = grid_sync(2 * nctas);  // every s_h row is written
-            ok = ok && g2;
+            // element): each epilogue warp stores the sum of the s_h values it wrote; after
+            // one grid barrier, Z_b = those totals of batch element b's CTAs summed in a
+            // fixed order, and s_l[t] = (sum_h s_h[h, t] in head order) / Z_b over this
+            // CTA's token range.
             const int cta = blockIdx.y * gridDim.x + blockIdx.x, Bn = gridDim.y / Hkv;
+            const int ew = warp - 4;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+            if (lane == 0) __stcg(norm_part + (size_t)cta * kEpiWarps + ew, zs);
+            const bool g2 = grid_sync(2 * nctas);  // every s_h row and warp total is stored
+            ok = ok && g2;
             const int cl = ceil_div(L, (int)nctas);
             const int t0 = min(L, cta * cl), t1 = min(L, t0 + cl);
-            const int ew = warp - 4;
+            const int per_b = (int)gridDim.x * Hkv * kEpiWarps;  // totals of one batch element
             for (int bb = 0; bb < Bn; ++bb) {
-                float ps = 0.0f;
+                float z = 0.0f;
+                if (ok)
+                    for (int e = et; e < per_b; e += kEpiWarps * 32)
+                        z += __ldcg(norm_part + (size_t)bb * per_b + e);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                if (lane == 0) sm.wsum[ew] = z;
+                named_barrier(1, kEpiWarps * 32);
+                float Z = 0.0f;
+                for (int w2 = 0; w2 < kEpiWarps; ++w2) Z += sm.wsum[w2];
                 if (ok)
                     for (int t = t0 + et; t < t1; t += kEpiWarps * 32) {
+                        const float *col = s_h + (size_t)bb * H * L + t;
                         float u = 0.0f;
-                        for (int h = 0; h < H; ++h) u += __ldcg(s_h + ((size_t)bb * H + h) * L + t);
-                        __stcg(s_l + (size_t)bb * L + t, u);
-                        ps += u;
+                        for (int h0 = 0; h0 < H; h0 += 32) {  // 32 heads' loads in flight
+                            float hv[32];
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)
+                                hv[k] = h0 + k < H ? __ldcg(col + (size_t)(h0 + k) * L) : 0.0f;
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)
+                                if (h0 + k < H) u += hv[k];
+                        }
+                        s_l[(size_t)bb * L + t] = u / Z;
                     }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-                if (lane == 0) sm.wsum[ew] = ps;
-                named_barrier(1, kEpiWarps * 32);
-                if (et == 0) {
-                    float z = 0.0f;
-                    for (int w2 = 0; w2 < kEpiWarps; ++w2) z += sm.wsum[w2];
-                    __stcg(norm_part + (size_t)bb * nctas + cta, z);
-                }
                 named_barrier(1, kEpiWarps * 32);  // wsum is free again
-            }
-            const bool g3 = grid_sync(3 * nctas);  // every partial sum is written
-            ok = ok && g3;
-            for (int bb = 0; bb < Bn; ++bb) {
-                if (ew == 0) {
-                    float z = 0.0f;
-                    for (int c = lane; c < (int)nctas; c += 32) z += __ldcg(norm_part + (size_t)bb * nctas + c);
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-                    if (lane == 0) sm.zsum = z;
-                }
-                named_barrier(1, kEpiWarps * 32);
-                const float Z = sm.zsum;
-                if (ok)
-                    for (int t = t0 + et; t < t1; t += kEpiWarps * 32)
-                        s_l[(size_t)bb * L + t] = __ldcg(s_l + (size_t)bb * L + t) / Z;
-                named_barrier(1, kEpiWarps * 32);  // zsum is free again
             }
         }
     }
@@ -507,6 +514,10 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
 cudaError_t launch_score_tc(const tsa_dims &dm, const void *Q, const void *K, int qe,
                             float scale, float *s_h, float *s_l, const WsLayout &w, char *ws,
                             cudaStream_t st, uint32_t limit_us, bool &fused) {
+    if (score_wave_eligible(dm, qe) && !force_single_wave()) {
+        fused = s_l != nullptr;
+        return launch_score_wave(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us);
+    }
     return dm.d == 64
                ? score_tc_impl<64>(dm, Q, K, qe, scale, s_h, s_l, w, ws, st, limit_us, fused)
                : score_tc_impl<128>(dm, Q, K, qe, scale, s_h, s_l, w, ws, st, limit_us, fused);

@@ -24,7 +24,7 @@ EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_b
            "tsa_select", "tsa_gather_qkv", "tsa_attn", "tsa_scatter_residual", "tsa_layer",
            "tsa_get_device_status", "tsa_set_wait_limit", "tsa_status_string",
            "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall",
-           "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex",
+           "tsa_set_score_schedule", "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex",
            "tsa_drift_workspace_size", "tsa_drift", "tsa_attn_gather",
            "tsa_block_workspace_size", "tsa_block_select", "tsa_attn_block")
 POOL_NONE, POOL_MAX, POOL_MEAN = 0, 1, 2
@@ -73,6 +73,7 @@ def lib():
             "tsa_get_device_status": (I32, [P, P]),
             "tsa_set_wait_limit": (None, [ctypes.c_uint32]),
             "tsa_set_test_stall": (None, [I32]),
+            "tsa_set_score_schedule": (None, [I32, I32]),
             "tsa_kernel_launches": (ctypes.c_uint64, []),
             "tsa_status_string": (ctypes.c_char_p, [I32]),
             "tsa_last_error": (ctypes.c_char_p, []),
@@ -378,3 +379,10 @@ def kernel_launches() -> int:
 def tsa_set_test_stall(on: bool):
     """Failure-path test hook (see include/tsa.h)."""
     lib().tsa_set_test_stall(1 if on else 0)
+
+
+def tsa_set_score_schedule(wave: bool, max_groups_per_wave: int = 0):
+    """bf16 scoring schedule: the single-wave kernel for every shape (False, the default)
+    or the wave-scheduled kernel where it applies (True); max_groups_per_wave > 0 caps
+    the KV groups of one wave.  See include/tsa.h."""
+    lib().tsa_set_score_schedule(1 if wave else 0, int(max_groups_per_wave))
