@@ -249,16 +249,6 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Per-warpgroup register budget: every thread of the warpgroup executes it.  The .inc
-// form draws on registers that .dec released elsewhere in the CTA, so the budgets must
-// add up to at most the launch's (threads x registers per thread).
-template <uint32_t N> __device__ __forceinline__ void setmaxnreg_inc() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N> __device__ __forceinline__ void setmaxnreg_dec() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // ---------------------------------------------------------------- math ---
 __device__ __forceinline__ float ex2(float x) {
     float y;
