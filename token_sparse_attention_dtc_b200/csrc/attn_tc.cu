@@ -235,7 +235,8 @@ __device__ __forceinline__ bool softmax_tile(AttnSmem<D> &sm, int X, int n, uint
         tmem_st32(tS + lo + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&sm.p_full[X]);
+        __syncwarp();  // every lane's P is in TMEM: one arrival per warp
+        if ((r & 31) == 0) mbar_arrive(&sm.p_full[X]);
     }
     l_out = l;
     return true;
@@ -295,7 +296,7 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&sm.s_full[x], 1);
-            mbar_init(&sm.p_full[x], 128);
+            mbar_init(&sm.p_full[x], 4);  // the 4 warps of the softmax warpgroup
             mbar_init(&sm.o_final[x], 1);
         }
         mbar_init(&sm.drain, 1);
