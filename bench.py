@@ -336,7 +336,8 @@ def run_ours(args, w, L, rank, world, local_rank):
     # ncu-counted DRAM bytes of the committed capture, when it matches the source
     for k, kern in (("score", "k_score_tc"), ("gather", "k_gather_qkv"),
                     ("scatter", "k_scatter_residual")):
-        t = _traffic(kern, w.name)
+        # the wave-scheduled scoring kernel has no committed capture of its own
+        t = None if (k == "score" and args.score_schedule != "single") else _traffic(kern, w.name)
         hbm_roof[k]["traffic"] = t
         hbm_roof[k]["dram_gbs"] = t / (stage_ms[k] * 1e-3) / 1e9 if t else None
         hbm_roof[k]["dram_frac"] = (t / (stage_ms[k] * 1e-3) / 1e9 / peaks["hbm"]) if t else None
@@ -532,7 +533,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "data": "synthetic",
             "config": {"workload": _workload_desc(w, L), "global_batch": world, "seq_len": L,
                        "parallelism": "replicas (dp%d, no data-path collective)" % world,
-                       "l2": l2_note(d),
+                       "l2": l2_note(d), "score_schedule": args.score_schedule,
                        "Lkeep": lk, "kept_fraction": lk / L},
             "roofline": roof,
             "stages_ms": stage_ms,
@@ -760,6 +761,8 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="tau x q sweep, B = 2, L = 64K")
     ap.add_argument("--drift", action="store_true",
                     help="drift pass on 32-layer Llama-8B-shaped calibration states")
+    ap.add_argument("--score-schedule", default="single", choices=("single", "wave"),
+                    help="bf16 scoring kernel: single-wave (default) or wave-scheduled")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
@@ -782,6 +785,10 @@ def main():
     if args.impl == "reference":  # rank 0 alone times the oracle; other ranks exit
         run_reference(args, w, L, rank, world)
         return
+    if args.score_schedule != "single":
+        from token_sparse_attention_dtc_b200 import tsa
+
+        tsa.tsa_set_score_schedule(True, 0)
     if world > 1:
         import datetime
 
