@@ -13,8 +13,8 @@
 // - Each CTA runs the phases P1(0), P1(1), P2(0), P1(2), P2(1), ..., P2(W-1).  The grid
 //   barrier that separates pass 1 and pass 2 of wave w (every CTA has stored its
 //   (max, sum) pairs of wave w and counted itself in) is waited for only after pass 1 of
-//   wave w+1, so it costs little idle time.  Each CTA then merges its group's pairs in
-//   split order itself (no CTA does the others' merge, so none falls behind).
+//   wave w+1, so it costs little idle time.  Each CTA then merges its group's pairs in a
+//   fixed order itself (no CTA does the others' merge, so none falls behind).
 // - Both passes compute S^T = Ktile * Qblk^T with the 128 tokens on the TMEM lanes and
 //   the N = 16*G query rows as columns (M = 128, N = 16*G).  Pass 1 therefore keeps a
 //   running (max, sum) per query row in every thread over the tokens of its lane, and
@@ -48,7 +48,7 @@ constexpr int kQSlots = 3;
 // which every CTA passes after its P2(w) merge has read the slot.
 constexpr int kPartSlots = 4;
 constexpr int kNbuf = 8, kLgb = 3, kBufCols = 64;  // TMEM ring: 8 x 64 columns
-constexpr int kMaxCtas = 160;  // scratch slots per wave (>= SMs of the part)
+constexpr int kMaxCtas = 160;  // pair slots per wave: the grid never exceeds 160 CTAs
 constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kNoMax = -1e30f;   // running max before any token (finite: no inf - inf)
 constexpr float kRescale = 8.0f;   // a value this far (log2 units) above the max moves it
@@ -65,7 +65,6 @@ template <int D> struct WaveSmem {
     int team_ok[4];           // pass 2: the team leader's barrier wait succeeded
     alignas(16) float mlog[kQRows];  // pass 2: max + log2(sum) per query row
     float wsum[kEpiWarps];   // layer score: per epilogue warp partial sums
-    float zsum;              // layer score: the batch element's total
     uint32_t tmem_base;
     int abort, never, flag_ok;
 };
@@ -99,8 +98,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_score_wave(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
              int L, int H, int Hkv, int Bn, int S, int gpw, int W, float sl2, float2 *part,
-             float *__restrict__ s_h, float *__restrict__ s_l, float *zp, unsigned int *sync, Control *ctl,
-             uint64_t limit_ns, int stall) {
+             float *__restrict__ s_h, float *__restrict__ s_l, float *zp, unsigned int *sync,
+             Control *ctl, uint64_t limit_ns, int stall) {
     extern __shared__ uint8_t smem_raw[];
     WaveSmem<D> &sm = *reinterpret_cast<WaveSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
