@@ -326,9 +326,9 @@ TSA_API void tsa_set_test_stall(int32_t on);
 
 /* Scoring schedule of bf16 inputs, for tests and measurements; default (0, 0).  With
  * wave = 0 every bf16 shape takes the single-wave kernel: every KV group at once, K read
- * from HBM twice (once per softmax pass).  With wave = 1, shapes of 16 recent queries
- * (q >= 16 and L >= 16) and at most 4 query heads per KV head take the wave-scheduled
- * kernel instead: the KV groups a few at a time (about 40 MB of K per wave), so that the
+ * from HBM twice (once per softmax pass).  With wave = 1, shapes whose recent-query
+ * count min(q, L) is 16, with at most 4 query heads per KV head and d = 64 or 128, take
+ * the wave-scheduled kernel instead: the KV groups a few at a time (about 40 MB of K per wave), so that the
  * second pass rereads K from L2 and K crosses HBM once.  The single-wave kernel is the
  * default because it is as fast or faster on one B200 at every length measured (the
  * wave schedule's tile pipeline is no faster from L2 than from HBM, and its passes run
