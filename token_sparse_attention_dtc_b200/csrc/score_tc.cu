@@ -21,9 +21,12 @@
 //   still in L2): S^T = Ktile · Qblk^T with the tokens on the TMEM lanes (N = query rows
 //   padded to 16).  Each thread owns one token and adds 2^(z2 - max_n) / sum_n over the
 //   rows of the heads of its column group in row order, then stores s_h[b, h, t].
-// Warp 0 streams K tiles by TMA through a 4-stage ring, warp 1 issues the MMAs into two
-// TMEM accumulators, warps 4-19 run the epilogue (4 TMEM lane quadrants x 4 column
-// groups).  The grid is at most one CTA per SM and is launched cooperatively, so every
+// Layer score (when one launch covers every group): each epilogue warp also sums the s_h
+//   values it wrote; after one more grid barrier, Z = those sums of the batch element's
+//   CTAs in a fixed order, and each CTA writes s_l = (sum over heads) / Z for its tokens.
+// Warp 0 streams K tiles by TMA through a 4-stage ring, warp 1 issues the MMAs into a
+// ring of TMEM accumulators (4 of 128 columns, or 2 of 256), warps 4-19 run the epilogue
+// (4 TMEM lane quadrants x 4 column groups).  The grid is at most one CTA per SM and is launched cooperatively, so every
 // CTA is resident for the grid barrier.  All waits are bounded.
 #include <math.h>
 
