@@ -173,35 +173,62 @@ def _staged(d, dm, Lk, idx):
 
 @pytest.mark.parametrize("B,L,H,Hkv,hd", [(1, 4096, 32, 8, 128), (2, 1000, 8, 2, 128),
                                            (2, 5000, 8, 8, 128), (2, 1500, 8, 2, 64)])
-def test_attn_gather_equals_staged_path_bitwise(B, L, H, Hkv, hd):
+def test_attn_gather_matches_oracle_and_staged_path(B, L, H, Hkv, hd):
+    """The fused compress + attention + decompress against the oracle (its selection
+    re-run on the GPU's scores, its attention on those indices), in place and out of
+    place, and bit for bit against the staged path."""
     x = make_inputs(B, L, H, Hkv, hd, torch.bfloat16, seed=L + H)
     d = {k: v.cuda() for k, v in x.items()}
     dm = tsa.dims(d["Q"], d["K"])
     s_h, s_l = tsa.tsa_score(d["Q"], d["K"], 16)
+    s_h_np = s_h.cpu().numpy()
     for keep in (None, [0] * B, [1] * B, [L] * B, [L // 3 + 7 * b for b in range(B)]):
         Lk = (tsa.tsa_budget(dm, s_l, 0.02) if keep is None
               else torch.tensor(keep, dtype=torch.int32, device="cuda"))
         idx = tsa.tsa_select(dm, s_h, Lk)
+        lk = Lk.cpu().numpy()
+        ref_idx = oracle.select(s_h_np, lk)
+        np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
         want = _staged(d, dm, Lk, idx)
         ws = tsa.workspace(dm, 1)
         got = tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, d["X"], ws=ws)
         Yi = d["X"].clone()
         tsa.tsa_attn_gather(d["Q"], d["K"], d["V"], idx, Lk, Yi, Yi, ws=ws)
         assert tsa.tsa_get_device_status(ws) == 0
+        _check_y(x, ref_idx, lk, got.cpu())
+        _check_y(x, ref_idx, lk, Yi.cpu())
         assert torch.equal(got, want), keep
         assert torch.equal(Yi, want), keep
         if keep is not None and keep[0] == 0:
             assert torch.equal(got, d["X"])
 
 
-def test_layer_direct_gather_equals_staged_layer():
+def test_layer_direct_gather_matches_oracle_and_staged_layer():
     x = make_inputs(2, 3000, 32, 8, 128, torch.bfloat16, seed=77)
     d = {k: v.cuda() for k, v in x.items()}
-    Y1 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, tau=0.01)
-    Y2 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, tau=0.01, direct=True)
-    Y3 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, sparsity=0.5, direct=True)
-    Y4 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, sparsity=0.5)
-    assert torch.equal(Y1, Y2) and torch.equal(Y3, Y4)
+    B, L, H = 2, 3000, 32
+    out = {}
+    for name, kw in (("tau", dict(tau=0.01)), ("fixed", dict(sparsity=0.5))):
+        s_h = torch.empty(B, H, L, device="cuda")
+        s_l = torch.empty(B, L, device="cuda")
+        Lk = torch.empty(B, dtype=torch.int32, device="cuda")
+        Y2 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, direct=True, s_h=s_h, s_l=s_l,
+                           Lkeep=Lk, **kw)
+        Y1 = tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, **kw)
+        assert torch.equal(Y1, Y2), name
+        g_sh, g_sl = s_h.cpu().numpy(), s_l.cpu().numpy()
+        ref_h, ref_l = oracle.score(x["Q"], x["K"], 16)
+        assert_scores_close(g_sh, ref_h, "s_h")
+        assert_scores_close(g_sl, ref_l, "s_l")
+        lk = (oracle.budget(g_sl, 0.01)[0] if name == "tau"
+              else oracle.budget_fixed(B, L, 0.5))
+        np.testing.assert_array_equal(Lk.cpu().numpy(), lk)
+        _check_y(x, oracle.select(g_sh, lk), lk, Y2.cpu())
+        out[name] = Y2
+    # in place: Y == X, the unselected segments untouched
+    Yi = d["X"].clone()
+    tsa.tsa_layer(d["Q"], d["K"], d["V"], Yi, Yi, q=16, tau=0.01, direct=True)
+    assert torch.equal(Yi, out["tau"])
 
 
 def test_attn_gather_reports_a_bad_index():

@@ -35,7 +35,7 @@ k_attn_simt(const T *__restrict__ Q, const T *__restrict__ K, const T *__restric
     const int ntiles = ceil_div(L, kBM);
     const int tile = ntiles - 1 - (int)(blockIdx.x / BH), bh = blockIdx.x % BH;
     const int b = bh / H, h = bh % H, kv = h / (H / Hkv);
-    const int Lk = dense ? L : Lkeep[b];
+    const int Lk = dense ? L : min(max(Lkeep[b], 0), L);  // clamped: rows past L untouched
     const int i0 = tile * kBM;
     if (i0 >= Lk) return;
     size_t qbase, kbase, qstride, kstride;

@@ -261,7 +261,11 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     const int ghead = min(hgroup, B_H - grp * hgroup);  // heads in this group
     const int bh = grp * hgroup + r % ghead, pair = npairs - 1 - r / ghead;
     const int b = bh / H, h = bh % H;
-    const int Lk = dense ? L : __ldg(Lkeep + b);
+    // A kept count outside [0, L] is clamped (and reported): rows past L are never
+    // read or written.
+    const int lk_in = dense ? L : __ldg(Lkeep + b);
+    const int Lk = min(max(lk_in, 0), L);
+    if (lk_in != Lk && pair == 0 && threadIdx.x == 0) report_error(ctl, TSA_ERR_INVALID_ARG, 30);
     const int i0 = pair * 2 * kBM;  // first row of tile A
     if (i0 >= Lk) return;
     const bool hasB = i0 + kBM < Lk;

@@ -30,7 +30,7 @@ k_block_means(const T *__restrict__ Qh, const T *__restrict__ Kh, const int32_t 
     constexpr int EPV = 16 / sizeof(T);  // elements per 16-byte load
     __shared__ float part[16][16 * EPV];
     const int bh = blockIdx.x, j = blockIdx.y, b = bh / H;
-    const int Lk = Lkeep[b];
+    const int Lk = min(max(Lkeep[b], 0), L);  // clamped: rows past L untouched
     const int rl = threadIdx.x / 16, cg = threadIdx.x % 16;
     const size_t base = (size_t)bh * L * d;
     auto mean_rows = [&](const T *src, int r0, int r1, float *dst) {
@@ -75,13 +75,13 @@ constexpr int kPairsPerCta = 32, kPairsPerWarp = kPairsPerCta / (kBlockThreads /
 
 __global__ void __launch_bounds__(kBlockThreads)
 k_block_select(const float *__restrict__ qbar, const float *__restrict__ kbar,
-               const int32_t *__restrict__ Lkeep, int H, int d, int NP, int NB, int NW,
+               const int32_t *__restrict__ Lkeep, int L, int H, int d, int NP, int NB, int NW,
                float scale, float theta, float *__restrict__ logits, uint32_t *__restrict__ mask) {
     extern __shared__ float4 sm4[];  // qs[kPairsPerCta][d], ks[32][d + 4] (16-byte aligned)
     float *qs = reinterpret_cast<float *>(sm4), *ks = qs + kPairsPerCta * d;
     const int kst = d + 4;  // 16-byte loads of 8 consecutive lanes hit distinct banks
     const int bh = blockIdx.y, b = bh / H, p0 = blockIdx.x * kPairsPerCta;
-    const int Lk = Lkeep[b];
+    const int Lk = min(max(Lkeep[b], 0), L);  // clamped: rows past L untouched
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int npair = max(0, min(kPairsPerCta, min(NP, ceil_div(Lk, 256)) - p0));
     for (int e = threadIdx.x; e < kPairsPerCta * d; e += kBlockThreads)
@@ -195,7 +195,7 @@ cudaError_t launch_block_select(const tsa_dims &dm, const void *Qh, const void *
         if (e != cudaSuccess) return e;
     }
     k_block_select<<<dim3(ceil_div(NP, kPairsPerCta), dm.B * dm.H), kBlockThreads, zsm, st>>>(
-        qbar, kbar, Lkeep, dm.H, dm.d, NP, NB, NW, scale, theta, logits, mask);
+        qbar, kbar, Lkeep, dm.L, dm.H, dm.d, NP, NB, NW, scale, theta, logits, mask);
     note_launches(2);
     return cudaGetLastError();
 }

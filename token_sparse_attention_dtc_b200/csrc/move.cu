@@ -23,7 +23,7 @@ k_gather_qkv(const uint4 *__restrict__ Q, const uint4 *__restrict__ K, const uin
              int Hkv, uint4 *__restrict__ Qh, uint4 *__restrict__ Kh, uint4 *__restrict__ Vh,
              Control *ctl) {
     const int bh = blockIdx.x, b = bh / H, h = bh % H, kv = h / (H / Hkv);
-    const int Lk = Lkeep[b];
+    const int Lk = min(max(Lkeep[b], 0), L);  // a count outside [0, L] is clamped
     const int pad_end = min(L, (Lk + 127) & ~127);
     const int i0 = blockIdx.y * kGatherRows;
     if (i0 >= pad_end) return;
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kMoveThreads)
 k_scatter_residual(const uint4 *__restrict__ Oh, const int32_t *__restrict__ idx,
                    const int32_t *__restrict__ Lkeep, const uint4 *X, uint4 *Y, int L, int H) {
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int Lk = Lkeep[b];
+    const int Lk = min(max(Lkeep[b], 0), L);  // a count outside [0, L] is clamped
     const int i0 = blockIdx.y * kGatherRows;
     const int iend = in_place ? Lk : L;
     if (i0 >= iend) return;
@@ -113,6 +113,7 @@ k_scatter_residual(const uint4 *__restrict__ Oh, const int32_t *__restrict__ idx
         const int i = i0 + e / VPR, v = e % VPR;
         if (i >= iend) break;
         const int t = S[i];
+        if ((unsigned)t >= (unsigned)L) continue;  // not a token of this sequence: skipped
         const size_t seg = (((size_t)b * L + t) * H + h) * VPR + v;
         const uint4 x = X[seg];
         if (i < Lk) Y[seg] = add_vec<T>(x, Oh[((size_t)bh * L + i) * VPR + v]);
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kMoveThreads)
 k_copy_rest(const int32_t *__restrict__ idx, const int32_t *__restrict__ Lkeep, const uint4 *X,
             uint4 *Y, int L, int H) {
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
-    const int Lk = Lkeep[b];
+    const int Lk = min(max(Lkeep[b], 0), L);
     const int i0 = max(blockIdx.y * kGatherRows, Lk), i1 = min(L, (blockIdx.y + 1) * kGatherRows);
     const int32_t *S = idx + (size_t)bh * L;
     for (int e = threadIdx.x; e < (i1 - i0) * VPR; e += kMoveThreads) {
