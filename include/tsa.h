@@ -31,7 +31,10 @@
  *            TSA_ERR_CUDA.  tsa_last_error() gives a message for the calling thread.
  *            Errors found on the device (a bounded wait that ran out, a score that is
  *            not a finite value in [0, 1]) are recorded in the workspace's error word
- *            and returned by tsa_get_device_status.
+ *            and returned by tsa_get_device_status.  The word keeps the first error
+ *            until it is read; after a device error, the results of later calls that
+ *            use the same workspace are undefined until tsa_get_device_status has
+ *            returned it (reading it also resets the workspace's grid-barrier words).
  *   Workspace `ws` is caller-owned device scratch of at least tsa_workspace_size()
  *            bytes (tsa_layer_workspace_size() for tsa_layer), 256-byte aligned,
  *            zero-filled once before its first use.  Calls that share a workspace
@@ -95,6 +98,36 @@ TSA_API tsa_status tsa_score(const tsa_dims *dims, const void *Q, const void *K,
                      float scale, float *s_h, float *s_l, void *ws, size_t ws_bytes,
                      void *stream);
 
+/* ---- One layer sharded by KV group across GPUs -------------------------------------- */
+/* [blog] §2.1 层级预算分配 and [notes] 关键设计 2: s_l is the normalised sum over all
+ * heads of s_h, so u[t] = sum_h s_h[h, t] is the only quantity that couples the heads.
+ * A GPU that holds a contiguous range of KV groups (its query heads, their K and V, and
+ * their columns of X and Y) runs:
+ *   tsa_score_partial        s_h of its heads and their unnormalised partial u;
+ *   an all-gather of every GPU's partial u (the caller's collective, e.g. NCCL);
+ *   tsa_layer_score_combine  the fixed-order sum of the gathered partials and s_l;
+ * then tsa_budget, tsa_select, tsa_gather_qkv, tsa_attn and tsa_scatter_residual on
+ * its own heads.  Every GPU combines the same partials in the same order, so s_l and
+ * L' are bit-identical on every GPU. */
+
+/* Scoring of this shard's heads: as tsa_score (dims, Q [B,L,H,d] and K [B,L,Hkv,d] are
+ * the shard's own: H and Hkv count its heads), writing s_h [B,H,L] and, in place of
+ * s_l, the partial layer score u_part[b,t] = sum over the shard's heads, in head order,
+ * of s_h[b,h,t] ([B,L] fp32, not normalised).  ws: tsa_workspace_size(dims, q) bytes. */
+TSA_API tsa_status tsa_score_partial(const tsa_dims *dims, const void *Q, const void *K,
+                                     int32_t q, float scale, float *s_h, float *u_part,
+                                     void *ws, size_t ws_bytes, void *stream);
+
+/* Layer score from the partials of nparts shards: u_parts [nparts, B, L] fp32 (shard r's
+ * u_part at u_parts + r*B*L; order them by rank), u[b,t] = sum over r = 0 .. nparts-1 in
+ * that order of u_parts[r,b,t], s_l[b,t] = u[b,t] / sum_t u[b,t] (the total in a fixed
+ * order).  Deterministic: the same partials give the same s_l bit for bit on every GPU.
+ * Only dims->B and dims->L are used (the other fields must be valid).  1 <= nparts <=
+ * 1024; s_l must not overlap u_parts.  ws: tsa_workspace_size(dims, 1) bytes. */
+TSA_API tsa_status tsa_layer_score_combine(const tsa_dims *dims, int32_t nparts,
+                                           const float *u_parts, float *s_l, void *ws,
+                                           size_t ws_bytes, void *stream);
+
 /* Coverage budget ([notes] 关键设计 2; [blog] §2.1 层级预算分配; [gist] §2 Budget
  * Allocation).  Sort s_l[b,:] ascending and find the smallest k whose cumulative mass
  * reaches tau; Lkeep[b] = L - k (k = L, so Lkeep = 0, if it is never reached).  The
@@ -117,7 +150,8 @@ TSA_API tsa_status tsa_select(const tsa_dims *dims, const float *s_h, const int3
  * Vh likewise.  Rows i in [Lkeep[b], min(L, ceil128(Lkeep[b]))) of Qh, Kh, Vh are
  * zero-filled (the attention kernel reads whole 128-row tiles); later rows are not
  * written.  An index outside [0, L) is skipped and reported as TSA_ERR_INVALID_ARG in the
- * workspace's error word (ws supplies only the error word). */
+ * workspace's error word (ws supplies only the error word).  Lkeep[b] outside [0, L] is
+ * clamped to that range. */
 TSA_API tsa_status tsa_gather_qkv(const tsa_dims *dims, const void *Q, const void *K,
                           const void *V, const int32_t *idx, const int32_t *Lkeep,
                           void *Qh, void *Kh, void *Vh, void *ws, size_t ws_bytes,
@@ -133,7 +167,9 @@ TSA_API tsa_status tsa_gather_qkv(const tsa_dims *dims, const void *Q, const voi
  * dense == 1: dense causal GQA attention of the full sequence (the pages' dense
  *   branch for layers outside the sparse set): Qh = Q [B,L,H,d], Kh = K and
  *   Vh = V [B,L,Hkv,d], Oh = O [B,L,H,d]; Lkeep is ignored and may be NULL.
- * scale > 0 (normally 1/sqrt(d)).  ws supplies the error word. */
+ * scale > 0 (normally 1/sqrt(d)).  ws supplies the error word.  A compressed-mode
+ * Lkeep[b] outside [0, L] is clamped to that range (no row at or past L is read or
+ * written) and reported as TSA_ERR_INVALID_ARG in the error word. */
 TSA_API tsa_status tsa_attn(const tsa_dims *dims, const void *Qh, const void *Kh, const void *Vh,
                     const int32_t *Lkeep, int32_t dense, float scale, void *Oh,
                     void *ws, size_t ws_bytes, void *stream);
@@ -147,7 +183,9 @@ TSA_API tsa_status tsa_attn(const tsa_dims *dims, const void *Qh, const void *Kh
  *     and only the kept segments are touched.
  *   idx == NULL: dense layer, Oh is O [B,L,H,d] and Y = X + O (Lkeep ignored).
  * The sum is formed in fp32 and rounded once to the output type.  Y may equal X;
- * no other aliasing is allowed. */
+ * no other aliasing is allowed.  Preconditions, enforced on the device without an error
+ * report (this call has no workspace): Lkeep[b] outside [0, L] is clamped to that range,
+ * and an index outside [0, L) is skipped, so no segment outside Y is written. */
 TSA_API tsa_status tsa_scatter_residual(const tsa_dims *dims, const void *Oh, const int32_t *idx,
                                 const int32_t *Lkeep, const void *X, void *Y, void *stream);
 
@@ -298,17 +336,35 @@ TSA_API tsa_status tsa_drift(int32_t n_layers, int64_t tokens, int32_t d_model, 
  *           that device current) and caches it; make that first call before any stream
  *           capture.
  *   Sharing every call on a device uses the same array, which keeps the last call's
- *           contents (the call clears the part that must start at zero).  Calls whose
- *           work overlaps on the GPU (other streams, or other host threads) race on it
- *           and must be serialised by the caller.  Device-side errors of this call are
- *           not readable through tsa_get_device_status.
+ *           contents; the scoring writes every scratch byte it reads before reading it.
+ *           Calls whose work overlaps on the GPU (other streams, or other host threads)
+ *           race on it and must be serialised by the caller.
+ *   Errors  device-side errors (a bounded wait that ran out) go to an error word in
+ *           the array, which keeps the first one until
+ *           tsa_score_fixed_scratch_status reads and clears it; until then the results
+ *           of later calls on that device are undefined.
+ *   Reset   the cached address belongs to the device's primary context; after
+ *           cudaDeviceReset (or another teardown of that context) call
+ *           tsa_score_fixed_scratch_forget() before calling again on that device.
  * It allocates and frees nothing. */
 TSA_API tsa_status tsa_score_fixed_scratch(const tsa_dims *dims, const void *Q, const void *K,
                                            int32_t q, float scale, float *s_h, float *s_l,
                                            void *stream);
 
+/* Device errors of tsa_score_fixed_scratch on the current device: synchronises
+ * `stream`, returns the error word of the fixed array (TSA_OK if none) and clears it
+ * (with the array's grid-barrier words, which a failed launch can leave part-way).
+ * Allocates nothing. */
+TSA_API tsa_status tsa_score_fixed_scratch_status(void *stream);
+
+/* Drops the cached device addresses of the fixed array on every device, so that the
+ * next tsa_score_fixed_scratch or tsa_score_fixed_scratch_status call on a device looks
+ * its address up again (needed after cudaDeviceReset).  Never fails. */
+TSA_API void tsa_score_fixed_scratch_forget(void);
+
 /* Synchronises `stream`, returns the device error word recorded in `ws` (TSA_OK if
- * none) and clears it. */
+ * none) and, if it is set, clears the 256-byte control block at the start of `ws` (the
+ * error word and the grid-barrier words). */
 TSA_API tsa_status tsa_get_device_status(void *ws, void *stream);
 
 /* Upper bound, in microseconds, of every device-side wait (on an mbarrier) in later

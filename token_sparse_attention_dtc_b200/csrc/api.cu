@@ -47,6 +47,8 @@ cudaError_t launch_attn_tc(const tsa_dims &, const void *, const void *, const v
                            uint32_t, const uint32_t * = nullptr);
 cudaError_t launch_scatter(const tsa_dims &, const void *, const int32_t *, const int32_t *,
                            const void *, void *, cudaStream_t);
+cudaError_t launch_head_sum(const tsa_dims &, const float *, float *, cudaStream_t);
+cudaError_t launch_combine_parts(int, int, int, const float *, float *, float *, cudaStream_t);
 
 static thread_local std::string g_last_error;
 static uint32_t g_wait_limit_us = 2000000;  // 2 s
@@ -234,6 +236,49 @@ tsa_status tsa_score(const tsa_dims *dims, const void *Q, const void *K, int32_t
     TSA_TRY(check_ptr(s_l, "s_l"));
     TSA_TRY(check_ws(ws, ws_bytes, ws_layout(*dims, q).total));
     return do_score(*dims, Q, K, q, scale, s_h, s_l, (char *)ws, (cudaStream_t)stream);
+}
+
+tsa_status tsa_score_partial(const tsa_dims *dims, const void *Q, const void *K, int32_t q,
+                             float scale, float *s_h, float *u_part, void *ws, size_t ws_bytes,
+                             void *stream) {
+    TSA_TRY(check_dims(dims));
+    TSA_TRY(check_q(dims, q));
+    TSA_TRY(check_scale(scale));
+    TSA_TRY(check_ptr(Q, "Q"));
+    TSA_TRY(check_ptr(K, "K"));
+    TSA_TRY(check_ptr(s_h, "s_h"));
+    TSA_TRY(check_ptr(u_part, "u_part"));
+    const tsa_dims &dm = *dims;
+    const WsLayout w = ws_layout(dm, q);
+    TSA_TRY(check_ws(ws, ws_bytes, w.total));
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    bool fused = false;  // no layer score here: s_l is not passed
+    if (dm.dtype == TSA_BF16)
+        e = launch_score_tc(dm, Q, K, w.qe, scale, s_h, nullptr, w, (char *)ws, st,
+                            g_wait_limit_us, fused);
+    else
+        e = launch_score_simt(dm, Q, K, w.qe, scale, s_h, w, (char *)ws, st);
+    TSA_TRY(cuda_status(e, "tsa_score_partial"));
+    return cuda_status(launch_head_sum(dm, s_h, u_part, st), "tsa_score_partial (head sum)");
+}
+
+tsa_status tsa_layer_score_combine(const tsa_dims *dims, int32_t nparts, const float *u_parts,
+                                   float *s_l, void *ws, size_t ws_bytes, void *stream) {
+    TSA_TRY(check_dims(dims));
+    if (nparts < 1 || nparts > 1024) return fail(TSA_ERR_INVALID_ARG, "nparts must be in [1, 1024]");
+    TSA_TRY(check_ptr(u_parts, "u_parts"));
+    TSA_TRY(check_ptr(s_l, "s_l"));
+    const size_t bytes = (size_t)4 * nparts * dims->B * dims->L;
+    const char *a = (const char *)u_parts, *o = (const char *)s_l;
+    if (a < o + (size_t)4 * dims->B * dims->L && o < a + bytes)
+        return fail(TSA_ERR_INVALID_ARG, "s_l overlaps u_parts");
+    const WsLayout w = ws_layout(*dims, 1);
+    TSA_TRY(check_ws(ws, ws_bytes, w.total));
+    return cuda_status(launch_combine_parts(dims->B, dims->L, nparts, u_parts, s_l,
+                                            (float *)((char *)ws + w.norm_part),
+                                            (cudaStream_t)stream),
+                       "tsa_layer_score_combine");
 }
 
 tsa_status tsa_budget(const tsa_dims *dims, const float *s_l, double tau, int32_t *Lkeep,
@@ -581,8 +626,10 @@ tsa_status tsa_get_device_status(void *ws, void *stream) {
     TSA_TRY(cuda_status(cudaMemcpy(&c, ws, sizeof c, cudaMemcpyDeviceToHost),
                         "tsa_get_device_status read"));
     if (c.err != 0) {
-        const int32_t zero[2] = {0, 0};
-        TSA_TRY(cuda_status(cudaMemcpy(ws, zero, sizeof zero, cudaMemcpyHostToDevice),
+        // The whole control block: the error word and the grid-barrier words, which a
+        // launch that failed part-way can leave off their initial state.
+        const Control zero{};
+        TSA_TRY(cuda_status(cudaMemcpy(ws, &zero, sizeof zero, cudaMemcpyHostToDevice),
                             "tsa_get_device_status clear"));
         return fail((tsa_status)c.err, "device error %d (detail %d)", c.err, c.err_where);
     }

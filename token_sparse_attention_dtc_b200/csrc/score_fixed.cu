@@ -25,18 +25,22 @@ static __device__ __align__(256) unsigned char g_score_scratch[kFixedScratchByte
 tsa_status set_error(tsa_status s, const char *msg);  // defined in api.cu
 
 // Device address of g_score_scratch on `dev`, looked up once per device (with that
-// device current) and cached.  Returns nullptr if the lookup fails.
+// device current) and cached.  Returns nullptr if the lookup fails.  The cached address
+// belongs to the device's current primary context: after cudaDeviceReset (or any other
+// teardown of that context) it is stale, and tsa_score_fixed_scratch_forget() must be
+// called before the next call on that device.
+static std::mutex g_mu;
+static void *g_addr[64] = {};
+
 static void *scratch_address(int dev) {
-    static std::mutex mu;
-    static void *addr[64] = {};
     if (dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_addr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_score_scratch) != cudaSuccess) return nullptr;
-        addr[dev] = p;
+        g_addr[dev] = p;
     }
-    return addr[dev];
+    return g_addr[dev];
 }
 
 }  // namespace tsa
@@ -64,11 +68,28 @@ extern "C" TSA_API tsa_status tsa_score_fixed_scratch(const tsa_dims *dims, cons
     if (!ws)
         return set_error(TSA_ERR_CUDA,
                          "tsa_score_fixed_scratch: cudaGetSymbolAddress of the scratch failed");
-    // The scratch keeps the previous call's contents.  Only the control block (the
-    // device error word) must start at zero; the scoring writes every other byte it
-    // reads before reading it.
-    const cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(Control), (cudaStream_t)stream);
-    if (e != cudaSuccess)
-        return set_error(TSA_ERR_CUDA, "tsa_score_fixed_scratch: clearing the scratch failed");
+    // The scratch keeps the previous call's contents.  The scoring writes every byte of
+    // it that it reads before reading it, and the grid barriers in the control block
+    // return to their initial state at the end of every launch that completes.  The
+    // device error word is sticky: it keeps the first error until
+    // tsa_score_fixed_scratch_status reads and clears it (which also resets the barriers
+    // a failed launch may have left part-way).
     return tsa_score(dims, Q, K, q, scale, s_h, s_l, ws, kFixedScratchBytes, stream);
+}
+
+extern "C" TSA_API tsa_status tsa_score_fixed_scratch_status(void *stream) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return set_error(TSA_ERR_CUDA, "tsa_score_fixed_scratch_status: cudaGetDevice failed");
+    void *ws = scratch_address(dev);
+    if (!ws)
+        return set_error(TSA_ERR_CUDA,
+                         "tsa_score_fixed_scratch_status: cudaGetSymbolAddress of the scratch "
+                         "failed");
+    return tsa_get_device_status(ws, stream);
+}
+
+extern "C" TSA_API void tsa_score_fixed_scratch_forget(void) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (void *&a : g_addr) a = nullptr;
 }

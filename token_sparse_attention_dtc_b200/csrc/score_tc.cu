@@ -26,8 +26,9 @@
 //   CTAs in a fixed order, and each CTA writes s_l = (sum over heads) / Z for its tokens.
 // Warp 0 streams K tiles by TMA through a 4-stage ring, warp 1 issues the MMAs into a
 // ring of TMEM accumulators (4 of 128 columns, or 2 of 256), warps 4-19 run the epilogue
-// (4 TMEM lane quadrants x 4 column groups).  The grid is at most one CTA per SM and is launched cooperatively, so every
-// CTA is resident for the grid barrier.  All waits are bounded.
+// (4 TMEM lane quadrants x 4 column groups).  The grid is at most one CTA per SM and is
+// launched cooperatively, so every CTA is resident for the grid barrier, whose word resets
+// itself (no memset between launches).  All waits are bounded.
 #include <math.h>
 
 #include <algorithm>
@@ -298,22 +299,29 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
                     online_merge(mm, ll, sm.red[g2][n].x, sm.red[g2][n].y);
                 __stcg(&part[((size_t)bg * nsplit + split) * N + n], make_float2(mm, ll));
             }
-        // Grid barrier among the epilogue warps of every CTA: the counter (zeroed before the
-        // launch) reaches `target` = nctas times the barrier's ordinal.  Every epilogue
-        // thread must call it (named barriers inside); it returns false when the wait ran
-        // out or the CTA aborted.
-        auto grid_sync = [&](unsigned target) -> bool {
+        // Grid barrier among the epilogue warps of every CTA, on a word that returns to its
+        // initial state by itself (no reset between launches): CTA 0 adds
+        // 2^31 - (nctas - 1), every other CTA adds 1, so bit 31 flips exactly when the
+        // last CTA arrives and the low 31 bits are back at zero.  A CTA waits until bit 31
+        // differs from the value its own add returned.  Every epilogue thread must call it
+        // (named barriers inside); it returns false when the wait ran out or the CTA
+        // aborted.  A launch that fails part-way can leave the word off its initial state:
+        // its error word is set, and reading the error (tsa_get_device_status) resets
+        // the control block.
+        const unsigned bar_add =
+            (blockIdx.x == 0 && blockIdx.y == 0) ? 0x80000000u - (nctas - 1u) : 1u;
+        auto grid_sync = [&]() -> bool {
             __threadfence();
             named_barrier(1, kEpiWarps * 32);
             if (et == 0) {
                 int good = 0;
                 if (!*abort) {
-                    atomicAdd(gbar, 1u);
+                    const unsigned old = atomicAdd(gbar, bar_add);
                     const uint64_t t0 = globaltimer_ns();
                     for (uint32_t k = 0;; ++k) {
                         unsigned v;
                         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gbar) : "memory");
-                        if (v >= target) { good = 1; break; }
+                        if ((v ^ old) & 0x80000000u) { good = 1; break; }
                         if ((k & 63) == 63 && (*abort || globaltimer_ns() - t0 > limit_ns)) break;
                         __nanosleep(64);
                     }
@@ -325,7 +333,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
         };
         // ---- grid barrier: every CTA's pass-1 pairs are in global memory
         {
-            const bool g1 = grid_sync(nctas);
+            const bool g1 = grid_sync();
             ok = ok && g1;
         }
         // ---- merge the pass-1 pairs of this group in split order: (max, 1/sum) per row
@@ -399,7 +407,7 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
             if (lane == 0) __stcg(norm_part + (size_t)cta * kEpiWarps + ew, zs);
-            const bool g2 = grid_sync(2 * nctas);  // every s_h row and warp total is stored
+            const bool g2 = grid_sync();  // every s_h row and warp total is stored
             ok = ok && g2;
             const int cl = ceil_div(L, (int)nctas);
             const int t0 = min(L, cta * cl), t1 = min(L, t0 + cl);
@@ -488,7 +496,8 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
     float sl2 = scale * 1.4426950408889634f;
     float2 *part = reinterpret_cast<float2 *>(ws + w.score_part);
     Control *ctl = reinterpret_cast<Control *>(ws);
-    unsigned int *gbar = reinterpret_cast<unsigned int *>(&ctl->pad[0]);
+    // pad[0..4] belong to the wave-scheduled kernel, which resets them before each launch.
+    unsigned int *gbar = reinterpret_cast<unsigned int *>(&ctl->pad[16]);
     uint64_t lim = (uint64_t)limit_us * 1000ull;
     int stall = test_stall();
     const __nv_bfloat16 *Qb = (const __nv_bfloat16 *)Q;
@@ -501,7 +510,6 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
     for (int g0 = 0; g0 < groups; g0 += per_launch) {
         int group0 = g0;
         const int gc = std::min(per_launch, groups - g0);
-        if ((e = cudaMemsetAsync(gbar, 0, sizeof(unsigned int), st))) return e;
         void *args[] = {&tk, (void *)&Qb, &L, &H, &Hkv, &qe, &sl2, &nsplit, &group0,
                         (void *)&part, (void *)&s_h, (void *)&sl, (void *)&np, (void *)&gbar,
                         (void *)&ctl, &lim, &stall};

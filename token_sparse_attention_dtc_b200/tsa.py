@@ -26,7 +26,9 @@ EXPORTS = ("tsa_workspace_size", "tsa_layer_workspace_size", "tsa_score", "tsa_b
            "tsa_last_error", "tsa_score_fixed_scratch", "tsa_set_test_stall",
            "tsa_set_score_schedule", "tsa_kernel_launches", "tsa_budget_fixed", "tsa_pool_scores", "tsa_layer_ex",
            "tsa_drift_workspace_size", "tsa_drift", "tsa_attn_gather",
-           "tsa_block_workspace_size", "tsa_block_select", "tsa_attn_block")
+           "tsa_block_workspace_size", "tsa_block_select", "tsa_attn_block",
+           "tsa_score_fixed_scratch_status", "tsa_score_fixed_scratch_forget",
+           "tsa_score_partial", "tsa_layer_score_combine")
 POOL_NONE, POOL_MAX, POOL_MEAN = 0, 1, 2
 BUDGET_COVERAGE, BUDGET_FIXED = 0, 1
 
@@ -65,6 +67,8 @@ def lib():
             "tsa_layer_workspace_size": (SZ, [DP, I32]),
             "tsa_score": (I32, [DP, P, P, I32, F, P, P, P, SZ, P]),
             "tsa_budget": (I32, [DP, P, D, P, P, SZ, P]),
+            "tsa_score_partial": (I32, [DP, P, P, I32, F, P, P, P, SZ, P]),
+            "tsa_layer_score_combine": (I32, [DP, I32, P, P, P, SZ, P]),
             "tsa_select": (I32, [DP, P, P, P, P, SZ, P]),
             "tsa_gather_qkv": (I32, [DP, P, P, P, P, P, P, P, P, P, SZ, P]),
             "tsa_attn": (I32, [DP, P, P, P, P, I32, F, P, P, SZ, P]),
@@ -78,6 +82,8 @@ def lib():
             "tsa_status_string": (ctypes.c_char_p, [I32]),
             "tsa_last_error": (ctypes.c_char_p, []),
             "tsa_score_fixed_scratch": (I32, [DP, P, P, I32, F, P, P, P]),
+            "tsa_score_fixed_scratch_status": (I32, [P]),
+            "tsa_score_fixed_scratch_forget": (None, []),
             "tsa_budget_fixed": (I32, [DP, D, P, P]),
             "tsa_attn_gather": (I32, [DP, P, P, P, P, P, F, P, P, P, SZ, P]),
             "tsa_block_workspace_size": (SZ, [DP]),
@@ -175,6 +181,42 @@ def tsa_score_fixed_scratch(Q, K, q: int, scale: float | None = None, s_h=None, 
                                          default_scale(dm.d) if scale is None else scale,
                                          _p(s_h), _p(s_l), _stream(stream)))
     return s_h, s_l
+
+
+def tsa_score_fixed_scratch_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the error word of the fixed scratch
+    on the current device."""
+    return int(lib().tsa_score_fixed_scratch_status(_stream(stream)))
+
+
+def tsa_score_partial(Q, K, q: int, scale: float | None = None, s_h=None, u_part=None,
+                      ws=None, stream=None):
+    """Scores of this shard's heads: returns (s_h [B, H, L], u_part [B, L]), u_part the
+    unnormalised sum of s_h over the shard's heads."""
+    dm = dims(Q, K)
+    _need_cuda(Q, K)
+    if s_h is None:
+        s_h = torch.empty(dm.B, dm.H, dm.L, dtype=torch.float32, device=Q.device)
+    if u_part is None:
+        u_part = torch.empty(dm.B, dm.L, dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = workspace(dm, q, device=Q.device)
+    _check(lib().tsa_score_partial(ctypes.byref(dm), _p(Q), _p(K), q,
+                                   default_scale(dm.d) if scale is None else scale, _p(s_h),
+                                   _p(u_part), _p(ws), ws.numel(), _stream(stream)))
+    return s_h, u_part
+
+
+def tsa_layer_score_combine(dm: Dims, u_parts, s_l=None, ws=None, stream=None):
+    """s_l [B, L] from the partials u_parts [nparts, B, L] (summed in index order)."""
+    _need_cuda(u_parts)
+    if s_l is None:
+        s_l = torch.empty(dm.B, dm.L, dtype=torch.float32, device=u_parts.device)
+    if ws is None:
+        ws = workspace(dm, 1, device=u_parts.device)
+    _check(lib().tsa_layer_score_combine(ctypes.byref(dm), int(u_parts.shape[0]), _p(u_parts),
+                                         _p(s_l), _p(ws), ws.numel(), _stream(stream)))
+    return s_l
 
 
 def tsa_budget(dm: Dims, s_l, tau: float, Lkeep=None, ws=None, stream=None):
