@@ -178,13 +178,37 @@ def _workload_desc(w, L):
 
 # --------------------------------------------------------------------------- oracle ---
 
-def oracle_sample(x, w, L, rows_per_sample=64, slice_div=64):
-    """Time the oracle on a bounded sample of one layer; return (ms per full layer, info)."""
+def host_cpu():
+    """Host cores the oracle may use and the CPU model (from /proc/cpuinfo)."""
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        usable = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return dict(nproc=usable, cpu_count=os.cpu_count(), model=model)
+
+
+def oracle_sample(x, w, L, attn_budget_s=30.0, slice_div=64):
+    """Time the oracle on one layer: scoring, budget and selection in full; attention on
+    whole heads when they fit in attn_budget_s (all of them at small L), else on a
+    strided sample of head 0's rows, extrapolated by exact causal pair count;
+    decompress + residual on 1/slice_div of the tokens, scaled by token count.  Returns
+    (ms per full layer, sample description, info, seconds spent)."""
     import numpy as np
 
     import oracle
 
-    threads = os.cpu_count() or 1
+    cpu = host_cpu()
+    threads = cpu["nproc"]
+    t_spent = time.perf_counter()
     t0 = time.perf_counter()
     s_h, s_l = oracle.score(x["Q"], x["K"], w.q, nthreads=threads)
     t1 = time.perf_counter()
@@ -193,33 +217,74 @@ def oracle_sample(x, w, L, rows_per_sample=64, slice_div=64):
     idx = oracle.select(s_h.astype(np.float32), lk)
     t3 = time.perf_counter()
     Lk = int(lk[0])
-    # attention: rows of head 0 spread over [0, L'), extrapolated by exact causal pair count
-    rows_i = sorted(set(np.linspace(0, max(Lk - 1, 0), rows_per_sample).astype(int).tolist()))
-    rows = [(0, 0, i) for i in rows_i] if Lk else []
-    ta = time.perf_counter()
-    if rows:
-        oracle.attend_rows(x["Q"], x["K"], x["V"], idx, lk, rows, nthreads=threads)
-    tb = time.perf_counter()
-    pairs_sample = sum(i + 1 for i in rows_i) if rows else 1
-    pairs_full = w.H * Lk * (Lk + 1) / 2
-    t_attn = (tb - ta) * pairs_full / pairs_sample if rows else 0.0
-    # decompress + residual on 1/slice_div of the tokens, scaled by token count
-    n = max(1, L // slice_div)
+    # attention: whole heads, one after another, while the next one is expected to fit in
+    # attn_budget_s (every head costs the same: each keeps L' rows); if even one head is
+    # not expected to fit (from a rate measured on 32 rows of head 0), every k-th row of
+    # head 0 instead
+    pairs_head = Lk * (Lk + 1) / 2.0
+    pairs_full = w.H * pairs_head
+    t_attn_meas, pairs_done, rows_timed, heads_done, stride = 0.0, 0.0, 0, 0, 0
+    if Lk:
+        cal = sorted(set(np.linspace(0, Lk - 1, 32).astype(int).tolist()))
+        tc0 = time.perf_counter()
+        oracle.attend_rows(x["Q"], x["K"], x["V"], idx, lk, [(0, 0, i) for i in cal],
+                           nthreads=threads)
+        rate = sum(i + 1 for i in cal) / max(time.perf_counter() - tc0, 1e-6)
+        if pairs_head / rate <= attn_budget_s:
+            per_head = pairs_head / rate
+            while heads_done < w.H and t_attn_meas + per_head <= attn_budget_s:
+                ta = time.perf_counter()
+                oracle.attend_rows(x["Q"], x["K"], x["V"], idx, lk,
+                                   [(0, heads_done, i) for i in range(Lk)], nthreads=threads)
+                per_head = time.perf_counter() - ta
+                t_attn_meas += per_head
+                heads_done += 1
+            pairs_done, rows_timed = heads_done * pairs_head, heads_done * Lk
+        else:
+            stride = max(2, int(math.ceil(pairs_head / max(attn_budget_s * rate, 1.0))))
+            rows_i = list(range(stride // 2, Lk, stride))
+            ta = time.perf_counter()
+            oracle.attend_rows(x["Q"], x["K"], x["V"], idx, lk, [(0, 0, i) for i in rows_i],
+                               nthreads=threads)
+            t_attn_meas = time.perf_counter() - ta
+            pairs_done, rows_timed = float(sum(i + 1 for i in rows_i)), len(rows_i)
+    factor = pairs_full / pairs_done if pairs_done else 1.0
+    t_attn = t_attn_meas * factor
+    # decompress + residual: in full while its fp64 arrays stay small (up to 2^25
+    # elements each), else on 1/slice_div of the tokens, scaled by token count
+    n = L if L * w.H * w.d <= (1 << 25) else max(1, L // slice_div)
     Oh = np.zeros((1, w.H, n, w.d))
     idx_s = np.tile(np.arange(n, dtype=np.int32), (1, w.H, 1))
-    tc = time.perf_counter()
+    td0 = time.perf_counter()
     oracle.decompress_residual(Oh, idx_s, np.array([min(Lk, n)], np.int32), x["X"][:, :n])
-    td = time.perf_counter()
-    t_dec = (td - tc) * L / n
+    td1 = time.perf_counter()
+    t_dec = (td1 - td0) * L / n
     total = (t1 - t0) + (t2 - t1) + (t3 - t2) + t_attn + t_dec
+    measured = (t1 - t0) + (t2 - t1) + (t3 - t2) + t_attn_meas + (td1 - td0)
+    if Lk == 0 or factor == 1.0:
+        attn_desc = "attention in full (%d heads x %d rows)" % (w.H, Lk)
+    elif heads_done:
+        attn_desc = ("attention on %d whole head(s) of %d (%d rows each), x%.4g by causal "
+                     "pair count" % (heads_done, w.H, Lk, factor))
+    else:
+        attn_desc = ("attention on every %d-th row of head 0 (%d of %d rows), x%.4g to all "
+                     "%d heads by causal pair count" % (stride, rows_timed, Lk, factor, w.H))
     info = dict(score_s=t1 - t0, budget_s=t2 - t1, select_s=t3 - t2,
-                attn_s_extrapolated=t_attn, attn_rows_sampled=len(rows),
-                decompress_s_extrapolated=t_dec, Lkeep=Lk, threads=threads)
-    sample = ("full scoring, budget and selection on the %d-token sequence; attention on %d "
-              "query rows of head 0 extrapolated to all %d heads by causal pair count; "
-              "decompress+residual on %d tokens scaled by token count"
-              % (L, len(rows), w.H, n))
-    return total * 1e3, sample, info, (tb - ta) + (t1 - t0) + (t2 - t1) + (t3 - t2) + (td - tc)
+                attn_s_measured=t_attn_meas, attn_extrapolation_factor=factor,
+                attn_s_extrapolated=t_attn, attn_rows_timed=rows_timed,
+                decompress_s_measured=td1 - td0, decompress_extrapolation_factor=L / n,
+                Lkeep=Lk, threads=threads, nproc=cpu["nproc"], cpu_count=cpu["cpu_count"],
+                cpu_model=cpu["model"], measured_s=measured,
+                measured_fraction=measured / total if total > 0 else 1.0,
+                wall_s=time.perf_counter() - t_spent)
+    dec_desc = ("decompress+residual in full" if n == L else
+                "decompress+residual on %d of %d tokens, x%d" % (n, L, L // n))
+    sample = ("scoring, budget and selection in full on the %d-token sequence; %s; %s; "
+              "%.3g%% of the layer's oracle time measured%s; %d threads on %s"
+              % (L, attn_desc, dec_desc, 100.0 * info["measured_fraction"],
+                 "" if info["measured_fraction"] >= 0.9999 else ", the rest extrapolated",
+                 threads, cpu["model"]))
+    return total * 1e3, sample, info, measured
 
 
 def run_reference(args, w, L, rank, world):
@@ -231,7 +296,8 @@ def run_reference(args, w, L, rank, world):
     times = []
     sample = info = None
     for s in range(args.warmup + args.steps):
-        ms, sample, info, _ = oracle_sample(x, w, L)
+        # each step a bounded sample: a few seconds of attention on the host cores
+        ms, sample, info, _ = oracle_sample(x, w, L, attn_budget_s=args.ref_attn_seconds)
         if s >= args.warmup:
             times.append(ms)
     v = statistics.mean(times)
@@ -242,7 +308,9 @@ def run_reference(args, w, L, rank, world):
         "data": "synthetic",
         "config": {"workload": _workload_desc(w, L), "oracle": "fp64 C, pthreads"},
         "cpu_baseline": {"value": v, "unit": "ms", "cores": info["threads"], "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "nproc": info["nproc"], "cpu_model": info["cpu_model"],
+                         "measured_fraction": info["measured_fraction"],
+                         "attn_extrapolation_factor": info["attn_extrapolation_factor"]},
         "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "oracle_breakdown_s": info,
     }
@@ -521,9 +589,12 @@ def run_ours(args, w, L, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ms, sample, info, _ = oracle_sample(x, w, L)
+        ms, sample, info, _ = oracle_sample(x, w, L, attn_budget_s=args.cpu_attn_seconds)
         cpu = {"value": ms, "unit": "ms", "cores": info["threads"], "kind": "oracle",
-               "sample": sample}
+               "sample": sample, "nproc": info["nproc"], "cpu_model": info["cpu_model"],
+               "measured_fraction": info["measured_fraction"],
+               "attn_extrapolation_factor": info["attn_extrapolation_factor"],
+               "breakdown_s": info}
 
     if rank == 0:
         line = {
@@ -755,6 +826,10 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-attn-seconds", type=float, default=30.0,
+                    help="host-core seconds of oracle attention in the cpu_baseline leg")
+    ap.add_argument("--ref-attn-seconds", type=float, default=3.0,
+                    help="host-core seconds of oracle attention per --impl reference step")
     ap.add_argument("--no-pages-sparsity", action="store_true")
     ap.add_argument("--stack", action="store_true",
                     help="32-layer stack with the sparse set chosen by the drift pass")
