@@ -32,6 +32,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "sm100.cuh"
 
@@ -454,16 +455,31 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
     }
 }
 
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
+}  // namespace
+
+// SM count of the current device, cached per device (the cooperative grid is sized from
+// it, so it must be the count of the device the launch goes to).
+int device_sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    if (dev < 0 || dev >= 64) {
+        int n = 0;
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+                       n > 0 ? n : 148;
+    }
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
             n = 148;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
     return n;
 }
+
+namespace {
+
+int sm_count() { return device_sm_count(); }
 
 }  // namespace
 

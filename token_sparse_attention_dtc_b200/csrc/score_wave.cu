@@ -37,6 +37,8 @@
 namespace tsa {
 using namespace sm100;
 
+int device_sm_count();  // score_tc.cu: SM count of the current device, cached per device
+
 namespace {
 
 constexpr int kThreads = 640, kStages = 5, kTile = 128, kQE = 16, kEpiWarps = 16;
@@ -558,16 +560,7 @@ k_score_wave(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     }
 }
 
-int wave_sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
-            n = 148;
-    }
-    return std::min(n, kMaxCtas);
-}
+int wave_sm_count() { return std::min(device_sm_count(), kMaxCtas); }
 
 }  // namespace
 
