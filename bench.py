@@ -62,6 +62,19 @@ def _traffic(kernel: str, workload: str):
     return e["bytes_per_launch"] if h == e["source_sha"] else None
 
 
+def score_kernel_name(schedule: str, w, L: int, B: int = 1, sms: int = 148) -> str:
+    """The bf16 scoring kernel the library runs for this schedule and shape (the rule of
+    tsa_set_score_schedule in include/tsa.h): the wave-scheduled kernel covers q_eff = 16,
+    at most 4 query heads per KV head and d = 64 or 128; the automatic schedule takes it
+    (every KV group in one wave) from 65536 tokens on, when B * Hkv fits the SMs."""
+    covered = (str(w.dtype) == "torch.bfloat16" and min(w.q, L) == 16 and w.H // w.Hkv <= 4
+               and w.d in (64, 128) and L >= 16)
+    if covered and (schedule == "wave" or
+                    (schedule == "auto" and L >= 65536 and B * w.Hkv <= min(sms, 160))):
+        return "k_score_wave"
+    return "k_score_tc" if str(w.dtype) == "torch.bfloat16" else "k_score_simt"
+
+
 def l2_note(d) -> str:
     """Whether the timed inputs exceed the 126 MB L2 (no flush is done between steps)."""
     mb = {k: d[k].numel() * d[k].element_size() / 1e6 for k in ("Q", "K", "V", "X")}
@@ -402,13 +415,51 @@ def run_ours(args, w, L, rank, world, local_rank):
                     "algorithmic_bytes": v}
                 for k, v in hbm.items()}
     # ncu-counted DRAM bytes of the committed capture, when it matches the source
-    for k, kern in (("score", "k_score_tc"), ("gather", "k_gather_qkv"),
+    score_kern = score_kernel_name(args.score_schedule, w, L)
+    for k, kern in (("score", score_kern), ("gather", "k_gather_qkv"),
                     ("scatter", "k_scatter_residual")):
-        # the wave-scheduled scoring kernel has no committed capture of its own
-        t = None if (k == "score" and args.score_schedule != "single") else _traffic(kern, w.name)
+        t = _traffic(kern, w.name)
         hbm_roof[k]["traffic"] = t
         hbm_roof[k]["dram_gbs"] = t / (stage_ms[k] * 1e-3) / 1e9 if t else None
         hbm_roof[k]["dram_frac"] = (t / (stage_ms[k] * 1e-3) / 1e9 / peaks["hbm"]) if t else None
+
+    # the scoring kernel on its own: the layer loop's score stage also absorbs the
+    # write-back of the previous scatter's dirty Y lines from L2 and the launch gap, so
+    # time the kernel after a flush that leaves L2 clean (a read of 512 MB after a write),
+    # with enough work queued ahead that the GPU never waits for the host
+    score_iso = None
+    if w.dtype == torch.bfloat16:
+        flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        s_h_i = torch.empty(1, w.H, L, device=dev)
+        s_l_i = torch.empty(1, L, device=dev)
+        ws_i = tsa.workspace(dm, w.q, device=dev)
+        for _ in range(3):
+            tsa.tsa_score(d["Q"], d["K"], w.q, s_h=s_h_i, s_l=s_l_i, ws=ws_i)
+        sync_all()
+        iso = []
+        for _ in range(max(5, args.steps)):
+            flush.zero_()
+            flush.view(torch.int32).max()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            tsa.tsa_score(d["Q"], d["K"], w.q, s_h=s_h_i, s_l=s_l_i, ws=ws_i)
+            b.record(st)
+            b.synchronize()
+            iso.append(a.elapsed_time(b))
+        if tsa.tsa_get_device_status(ws_i) != 0:
+            raise RuntimeError("device error in the isolated scoring runs")
+        score_iso = statistics.median(iso)
+        del flush, s_h_i, s_l_i, ws_i
+
+    if score_iso is not None:
+        v = hbm["score"]
+        hbm_roof["score"]["kernel_ms_isolated"] = score_iso
+        hbm_roof["score"]["isolated_achieved_gbs"] = v / (score_iso * 1e-3) / 1e9
+        hbm_roof["score"]["isolated_frac"] = v / (score_iso * 1e-3) / 1e9 / peaks["hbm"]
+        t = hbm_roof["score"].get("traffic")
+        if t:
+            hbm_roof["score"]["isolated_dram_frac"] = t / (score_iso * 1e-3) / 1e9 / peaks["hbm"]
 
     # dense causal attention through the same kernel, same shape
     dense = None
@@ -605,6 +656,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "config": {"workload": _workload_desc(w, L), "global_batch": world, "seq_len": L,
                        "parallelism": "replicas (dp%d, no data-path collective)" % world,
                        "l2": l2_note(d), "score_schedule": args.score_schedule,
+                       "score_kernel": score_kern,
                        "Lkeep": lk, "kept_fraction": lk / L},
             "roofline": roof,
             "stages_ms": stage_ms,
@@ -836,8 +888,9 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="tau x q sweep, B = 2, L = 64K")
     ap.add_argument("--drift", action="store_true",
                     help="drift pass on 32-layer Llama-8B-shaped calibration states")
-    ap.add_argument("--score-schedule", default="single", choices=("single", "wave"),
-                    help="bf16 scoring kernel: single-wave (default) or wave-scheduled")
+    ap.add_argument("--score-schedule", default="auto", choices=("auto", "single", "wave"),
+                    help="bf16 scoring kernel: the library's automatic choice (default), the "
+                         "single-wave kernel everywhere, or the wave-scheduled kernel")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
@@ -860,10 +913,10 @@ def main():
     if args.impl == "reference":  # rank 0 alone times the oracle; other ranks exit
         run_reference(args, w, L, rank, world)
         return
-    if args.score_schedule != "single":
+    if args.score_schedule != "auto":
         from token_sparse_attention_dtc_b200 import tsa
 
-        tsa.tsa_set_score_schedule(True, 0)
+        tsa.tsa_set_score_schedule(1 if args.score_schedule == "wave" else "single", 0)
     if world > 1:
         import datetime
 

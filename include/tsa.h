@@ -380,18 +380,24 @@ TSA_API void tsa_set_wait_limit(uint32_t microseconds);
  * down as described above, and exits.  Nothing faults, traps or hangs. */
 TSA_API void tsa_set_test_stall(int32_t on);
 
-/* Scoring schedule of bf16 inputs, for tests and measurements; default (0, 0).  With
- * wave = 0 every bf16 shape takes the single-wave kernel: every KV group at once, K read
- * from HBM twice (once per softmax pass).  With wave = 1, shapes whose recent-query
- * count min(q, L) is 16, with at most 4 query heads per KV head and d = 64 or 128, take
- * the wave-scheduled kernel instead: the KV groups a few at a time (about 40 MB of K per wave), so that the
- * second pass rereads K from L2 and K crosses HBM once.  The single-wave kernel is the
- * default because it is as fast or faster on one B200 at every length measured (the
- * wave schedule's tile pipeline is no faster from L2 than from HBM, and its passes run
- * one after the other).  max_groups_per_wave > 0 caps the groups of one wave (more
- * waves on small inputs); 0 lets the library choose.  Both kernels give the scores
- * tsa_score defines, within fp32 rounding; they differ in summation order only.
- * Applies to later launches from any thread. */
+/* Scoring schedule of bf16 inputs, for tests and measurements; default (0, 0).  Two
+ * kernels compute the same exact two-pass scores, within fp32 rounding (they differ in
+ * summation order only):
+ *   the single-wave kernel: every KV group at once; pass 1 with the recent-query rows on
+ *     the TMEM lanes, pass 2 with the tokens on the lanes; K read from HBM twice;
+ *   the wave-scheduled kernel: shapes whose recent-query count min(q, L) is 16, with at
+ *     most 4 query heads per KV head and d = 64 or 128; tokens on the TMEM lanes in both
+ *     passes; the KV groups in waves (one wave, or a few groups per wave so that pass 2
+ *     rereads K from L2).
+ * wave = 0 (automatic, the default): the wave-scheduled kernel with every KV group in one
+ *   wave for the shapes it covers with L >= 65536 tokens and B * Hkv no more than the
+ *   SMs, else the single-wave kernel (measured on one B200: the one-wave schedule is
+ *   about 12% faster at 64K-128K tokens, equal at 32K, slower at 4K).
+ * wave = 1: the wave-scheduled kernel for every shape it covers, about 40 MB of K per
+ *   wave; max_groups_per_wave > 0 caps the groups of one wave (more waves on small
+ *   inputs), 0 lets the library choose.
+ * wave = 2: the single-wave kernel for every shape.
+ * Other values act as 0.  Applies to later launches from any thread. */
 TSA_API void tsa_set_score_schedule(int32_t wave, int32_t max_groups_per_wave);
 
 /* Number of CUDA kernels this library has launched in this process, on every device and

@@ -1,14 +1,17 @@
-"""The two tensor-core scoring schedules against the oracle, through the C ABI.
+"""The two tensor-core scoring kernels against the oracle, through the C ABI.
 
-The wave-scheduled kernel (opt-in) scores the KV groups a few at a time (pass 1 of wave
-w+1 runs before pass 2 of wave w; each CTA merges its group's statistics after a per-wave
-count); the single-wave kernel (the default) scores every group at once.  Both must give s_h and s_l within the
+The wave-scheduled kernel scores the KV groups in waves (pass 1 of wave w+1 runs before
+pass 2 of wave w; each CTA merges its group's statistics after a per-wave count); the
+single-wave kernel scores every group at once.  The automatic schedule (the default)
+takes the wave-scheduled kernel with every group in one wave from 65536 tokens on, and
+the single-wave kernel below.  Every kernel and plan must give s_h and s_l within the
 scoring tolerance (relative 1e-5) of the oracle on the same inputs, on shapes that cover:
 - one wave, two waves, and many waves (the two statistics slots reused);
 - a ragged last tile, the shortest eligible sequence (16 tokens, one tile), and a tile
   holding a single token;
 - 1, 2 and 4 query heads per KV head (idle epilogue warps when fewer than 4);
-- d = 64 and 128, batches of 1 to 20 sequences (160 KV groups in one launch).
+- d = 64 and 128, batches of 1 to 20 sequences (160 KV groups in one launch);
+- the automatic one-wave plan at 64K+ tokens (a ragged tail, and two sequences).
 """
 import numpy as np
 import pytest
@@ -37,7 +40,7 @@ class schedule:
         tsa.tsa_set_score_schedule(self.wave, self.cap)
 
     def __exit__(self, *a):
-        tsa.tsa_set_score_schedule(False, 0)  # the default
+        tsa.tsa_set_score_schedule(0, 0)  # the default: automatic
 
 
 # (B, L, H, Hkv, d, groups-per-wave cap): the comment gives the wave plan on 148 SMs
@@ -59,7 +62,7 @@ def test_wave_and_single_wave_scoring_match_the_oracle(B, L, H, Hkv, d, cap):
     Q, K = x["Q"].cuda(), x["K"].cuda()
     ref_h, ref_l = oracle.score(x["Q"], x["K"], 16)
     out = {}
-    for wave in (True, False):
+    for wave in (True, "single"):
         with schedule(wave, cap):
             s_h, s_l = tsa.tsa_score(Q, K, 16)
             torch.cuda.synchronize()
@@ -67,7 +70,7 @@ def test_wave_and_single_wave_scoring_match_the_oracle(B, L, H, Hkv, d, cap):
         _close(s_l.cpu().numpy(), ref_l, "s_l wave=%s" % wave)
         out[wave] = (s_h, s_l)
     # the two schedules agree with each other to fp32 summation order
-    for a, b in zip(out[True], out[False]):
+    for a, b in zip(out[True], out["single"]):
         np.testing.assert_allclose(a.cpu().numpy(), b.cpu().numpy(), rtol=1e-5, atol=1e-30)
 
 
@@ -97,3 +100,22 @@ def test_wave_scoring_inside_a_layer_matches_the_oracle():
     ref_h, ref_l = oracle.score(x["Q"], x["K"], 16)
     _close(s_h.cpu().numpy(), ref_h, "s_h in a layer")
     _close(s_l.cpu().numpy(), ref_l, "s_l in a layer")
+
+
+@pytest.mark.parametrize("B,L,H,Hkv", [(1, 65536 + 37, 32, 8), (2, 65536, 16, 4)])
+def test_automatic_one_wave_schedule_matches_the_oracle(B, L, H, Hkv):
+    """From 65536 tokens on the default schedule scores every KV group in one wave of the
+    wave-scheduled kernel; it matches the oracle and the single-wave kernel, and repeated
+    launches are bit-identical."""
+    x = make_inputs(B, L, H, Hkv, 128, torch.bfloat16, seed=L + B)
+    Q, K = x["Q"].cuda(), x["K"].cuda()
+    ref_h, ref_l = oracle.score(x["Q"], x["K"], 16)
+    s_h, s_l = tsa.tsa_score(Q, K, 16)                  # automatic
+    _close(s_h.cpu().numpy(), ref_h, "s_h one wave")
+    _close(s_l.cpu().numpy(), ref_l, "s_l one wave")
+    again = tsa.tsa_score(Q, K, 16)
+    assert torch.equal(again[0], s_h) and torch.equal(again[1], s_l)
+    with schedule("single"):
+        u_h, u_l = tsa.tsa_score(Q, K, 16)
+    _close(u_h.cpu().numpy(), ref_h, "s_h single wave")
+    np.testing.assert_allclose(s_l.cpu().numpy(), u_l.cpu().numpy(), rtol=1e-5, atol=1e-30)

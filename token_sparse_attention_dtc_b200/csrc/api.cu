@@ -56,7 +56,7 @@ static int g_test_stall = 0;
 static int g_score_wave = 0, g_score_wave_cap = 0;
 
 int test_stall() { return g_test_stall; }
-bool force_single_wave() { return g_score_wave == 0; }  // the default
+int score_schedule() { return g_score_wave; }  // 0 = automatic (the default)
 int score_wave_group_cap() { return g_score_wave_cap; }
 
 static std::atomic<uint64_t> g_launches{0};
@@ -641,7 +641,7 @@ void tsa_set_wait_limit(uint32_t microseconds) { g_wait_limit_us = microseconds;
 void tsa_set_test_stall(int32_t on) { g_test_stall = on ? 1 : 0; }
 
 void tsa_set_score_schedule(int32_t wave, int32_t max_groups_per_wave) {
-    g_score_wave = wave ? 1 : 0;
+    g_score_wave = (wave == 1 || wave == 2) ? wave : 0;
     g_score_wave_cap = max_groups_per_wave > 0 ? max_groups_per_wave : 0;
 }
 

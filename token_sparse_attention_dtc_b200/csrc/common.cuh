@@ -129,9 +129,9 @@ inline int score_split_cap(const tsa_dims &dm) {
 
 // Host: the failure-path test hook set by tsa_set_test_stall (0 or 1).
 int test_stall();
-// Host: true (the default) unless tsa_set_score_schedule(1, ...) lets the shapes it
-// covers take the wave-scheduled scoring kernel.
-bool force_single_wave();
+// Host: the scoring schedule set by tsa_set_score_schedule: 0 automatic (the default),
+// 1 the wave-scheduled kernel wherever it applies, 2 the single-wave kernel everywhere.
+int score_schedule();
 // Host: the cap on KV groups per wave set by tsa_set_score_schedule (0: none).
 int score_wave_group_cap();
 

@@ -41,9 +41,15 @@ using namespace sm100;
 
 // The wave-scheduled kernel (score_wave.cu) takes the shapes it covers.
 bool score_wave_eligible(const tsa_dims &dm, int qe);
+bool score_one_wave_fits(const tsa_dims &dm);
 cudaError_t launch_score_wave(const tsa_dims &dm, const void *Q, const void *K, float scale,
                               float *s_h, float *s_l, const WsLayout &w, char *ws,
-                              cudaStream_t st, uint32_t limit_us);
+                              cudaStream_t st, uint32_t limit_us, bool one_wave);
+
+// From this many tokens on, the automatic schedule scores every KV group in one wave of the
+// wave-scheduled kernel (tokens on the TMEM lanes in both passes); below it, the
+// single-wave kernel here is as fast or faster.
+constexpr int kOneWaveMinTokens = 65536;
 
 namespace {
 
@@ -541,9 +547,13 @@ static cudaError_t score_tc_impl(const tsa_dims &dm, const void *Q, const void *
 cudaError_t launch_score_tc(const tsa_dims &dm, const void *Q, const void *K, int qe,
                             float scale, float *s_h, float *s_l, const WsLayout &w, char *ws,
                             cudaStream_t st, uint32_t limit_us, bool &fused) {
-    if (score_wave_eligible(dm, qe) && !force_single_wave()) {
-        fused = s_l != nullptr;
-        return launch_score_wave(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us);
+    const int mode = score_schedule();
+    if (score_wave_eligible(dm, qe)) {
+        const bool one = mode == 0 && dm.L >= kOneWaveMinTokens && score_one_wave_fits(dm);
+        if (mode == 1 || one) {
+            fused = s_l != nullptr;
+            return launch_score_wave(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us, one);
+        }
     }
     return dm.d == 64
                ? score_tc_impl<64>(dm, Q, K, qe, scale, s_h, s_l, w, ws, st, limit_us, fused)

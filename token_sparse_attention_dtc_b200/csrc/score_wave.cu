@@ -571,12 +571,23 @@ bool score_wave_eligible(const tsa_dims &dm, int qe) {
     return true;
 }
 
-// The wave plan: gpw groups per wave (the largest divisor of B*Hkv with at most ~40 MB of
-// K per wave and, when there are two or more groups, at least two waves), S splits per
-// group, gpw * S <= SMs CTAs.
-void score_wave_plan(const tsa_dims &dm, int &gpw, int &S, int &W) {
+// Every KV group in one wave: one CTA per split of every group, so at most one group
+// per SM.
+bool score_one_wave_fits(const tsa_dims &dm) { return dm.B * dm.Hkv <= wave_sm_count(); }
+
+// The wave plan.  one_wave: every group in one wave (gpw = B*Hkv, W = 1).  Otherwise gpw
+// groups per wave (the largest divisor of B*Hkv with at most ~40 MB of K per wave and,
+// when there are two or more groups, at least two waves).  S splits per group,
+// gpw * S <= SMs CTAs.
+void score_wave_plan(const tsa_dims &dm, bool one_wave, int &gpw, int &S, int &W) {
     const int groups = dm.B * dm.Hkv, sms = wave_sm_count();
     const int ntiles = ceil_div(dm.L, kTile);
+    if (one_wave) {
+        gpw = groups;
+        S = std::max(1, std::min(ntiles, sms / gpw));
+        W = 1;
+        return;
+    }
     const double kg = (double)dm.L * dm.d * 2.0;
     int cap = (int)std::max(1.0, (40.0 * (1 << 20)) / kg);
     cap = std::min(cap, std::max(1, groups / 2));
@@ -595,7 +606,8 @@ void score_wave_plan(const tsa_dims &dm, int &gpw, int &S, int &W) {
 template <int D>
 static cudaError_t score_wave_impl(const tsa_dims &dm, const void *Q, const void *K,
                                    float scale, float *s_h, float *s_l, const WsLayout &w,
-                                   char *ws, cudaStream_t st, uint32_t limit_us) {
+                                   char *ws, cudaStream_t st, uint32_t limit_us,
+                                   bool one_wave) {
     CUtensorMap tk;
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)dm.L, (uint64_t)dm.Hkv, (uint64_t)dm.B};
     const uint64_t strides[3] = {(uint64_t)dm.Hkv * D * 2, (uint64_t)D * 2,
@@ -614,7 +626,7 @@ static cudaError_t score_wave_impl(const tsa_dims &dm, const void *Q, const void
                                   (int)smem)))
         return e;
     int gpw, S, W;
-    score_wave_plan(dm, gpw, S, W);
+    score_wave_plan(dm, one_wave, gpw, S, W);
     float sl2 = scale * 1.4426950408889634f;
     float2 *part = reinterpret_cast<float2 *>(ws + w.score_part);
     Control *ctl = reinterpret_cast<Control *>(ws);
@@ -633,12 +645,14 @@ static cudaError_t score_wave_impl(const tsa_dims &dm, const void *Q, const void
     return e;
 }
 
-// Scoring with the wave schedule; s_l may be NULL (s_h only).
+// Scoring with the wave schedule (one_wave: every group in one wave); s_l may be NULL
+// (s_h only).
 cudaError_t launch_score_wave(const tsa_dims &dm, const void *Q, const void *K, float scale,
                               float *s_h, float *s_l, const WsLayout &w, char *ws,
-                              cudaStream_t st, uint32_t limit_us) {
-    return dm.d == 64 ? score_wave_impl<64>(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us)
-                      : score_wave_impl<128>(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us);
+                              cudaStream_t st, uint32_t limit_us, bool one_wave) {
+    return dm.d == 64
+               ? score_wave_impl<64>(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us, one_wave)
+               : score_wave_impl<128>(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us, one_wave);
 }
 
 }  // namespace tsa

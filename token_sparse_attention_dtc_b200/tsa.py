@@ -423,8 +423,10 @@ def tsa_set_test_stall(on: bool):
     lib().tsa_set_test_stall(1 if on else 0)
 
 
-def tsa_set_score_schedule(wave: bool, max_groups_per_wave: int = 0):
-    """bf16 scoring schedule: the single-wave kernel for every shape (False, the default)
-    or the wave-scheduled kernel where it applies (True); max_groups_per_wave > 0 caps
-    the KV groups of one wave.  See include/tsa.h."""
-    lib().tsa_set_score_schedule(1 if wave else 0, int(max_groups_per_wave))
+def tsa_set_score_schedule(wave, max_groups_per_wave: int = 0):
+    """bf16 scoring schedule: 0 / False the automatic choice (the default), 1 / True the
+    wave-scheduled kernel wherever it applies, 2 / "single" the single-wave kernel
+    everywhere; max_groups_per_wave > 0 caps the KV groups of one wave.  See
+    include/tsa.h."""
+    mode = 2 if wave == "single" else (1 if wave is True else int(wave))
+    lib().tsa_set_score_schedule(mode, int(max_groups_per_wave))
