@@ -66,11 +66,13 @@ def score_kernel_name(schedule: str, w, L: int, B: int = 1, sms: int = 148) -> s
     """The bf16 scoring kernel the library runs for this schedule and shape (the rule of
     tsa_set_score_schedule in include/tsa.h): the wave-scheduled kernel covers q_eff = 16,
     at most 4 query heads per KV head and d = 64 or 128; the automatic schedule takes it
-    (every KV group in one wave) from 65536 tokens on, when B * Hkv fits the SMs."""
+    (every KV group in one wave) when K holds at least 192 MiB and B * Hkv fits the SMs."""
     covered = (str(w.dtype) == "torch.bfloat16" and min(w.q, L) == 16 and w.H // w.Hkv <= 4
                and w.d in (64, 128) and L >= 16)
+    kbytes = 2.0 * B * L * w.Hkv * w.d
     if covered and (schedule == "wave" or
-                    (schedule == "auto" and L >= 65536 and B * w.Hkv <= min(sms, 160))):
+                    (schedule == "auto" and kbytes >= 192.0 * (1 << 20)
+                     and B * w.Hkv <= min(sms, 160))):
         return "k_score_wave"
     return "k_score_tc" if str(w.dtype) == "torch.bfloat16" else "k_score_simt"
 
@@ -866,6 +868,57 @@ def run_drift(args):
         del h, ws
 
 
+def run_score_only(args, w, L):
+    """The scoring kernel alone (tsa_score: s_h and the layer score) on the workload's Q
+    and K, each launch after an L2 flush that leaves L2 clean; one JSON line with the HBM
+    roofline by algorithmic bytes.  Allocates only Q, K, s_h, s_l and the workspace, so a
+    profiler capture of it stays small."""
+    import torch
+
+    from token_sparse_attention_dtc_b200 import tsa
+    from token_sparse_attention_dtc_b200.inputs import make_workload
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    x = make_workload(w.name, seed=args.seed, L=L, B=1)
+    Q, K = x["Q"].to(dev), x["K"].to(dev)
+    del x
+    dm = tsa.dims(Q, K)
+    ws = tsa.workspace(dm, w.q, device=dev)
+    s_h = torch.empty(1, w.H, L, device=dev)
+    s_l = torch.empty(1, L, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream(dev)
+    for _ in range(max(args.warmup, 3)):
+        tsa.tsa_score(Q, K, w.q, s_h=s_h, s_l=s_l, ws=ws)
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        flush.view(torch.int32).max()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        tsa.tsa_score(Q, K, w.q, s_h=s_h, s_l=s_l, ws=ws)
+        b.record(st)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    if tsa.tsa_get_device_status(ws) != 0:
+        raise RuntimeError("device error in the scoring runs")
+    ms = statistics.median(ts)
+    nbytes = L * w.Hkv * w.d * 2 + w.q * w.H * w.d * 2 + 4 * w.H * L + 4 * L
+    pk = _peaks()
+    kern = score_kernel_name(args.score_schedule, w, L)
+    print(json.dumps({
+        "metric": "scoring kernel ms (tsa_score: s_h and s_l)", "value": ms, "unit": "ms",
+        "higher_is_better": False, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": _workload_desc(w, L), "score_kernel": kern,
+                   "l2": "L2 flushed (512 MB written, then read) before each launch"},
+        "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm"],
+                     "traffic": _traffic(kern, w.name), "algorithmic_bytes": nbytes}}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -886,6 +939,8 @@ def main():
     ap.add_argument("--stack", action="store_true",
                     help="32-layer stack with the sparse set chosen by the drift pass")
     ap.add_argument("--sweep", action="store_true", help="tau x q sweep, B = 2, L = 64K")
+    ap.add_argument("--score-only", action="store_true",
+                    help="time the scoring kernel alone on the workload (L2 flushed per launch)")
     ap.add_argument("--drift", action="store_true",
                     help="drift pass on 32-layer Llama-8B-shaped calibration states")
     ap.add_argument("--score-schedule", default="auto", choices=("auto", "single", "wave"),
@@ -917,6 +972,9 @@ def main():
         from token_sparse_attention_dtc_b200 import tsa
 
         tsa.tsa_set_score_schedule(1 if args.score_schedule == "wave" else "single", 0)
+    if args.score_only:
+        run_score_only(args, w, L)
+        return
     if world > 1:
         import datetime
 

@@ -390,9 +390,10 @@ TSA_API void tsa_set_test_stall(int32_t on);
  *     passes; the KV groups in waves (one wave, or a few groups per wave so that pass 2
  *     rereads K from L2).
  * wave = 0 (automatic, the default): the wave-scheduled kernel with every KV group in one
- *   wave for the shapes it covers with L >= 65536 tokens and B * Hkv no more than the
- *   SMs, else the single-wave kernel (measured on one B200: the one-wave schedule is
- *   about 12% faster at 64K-128K tokens, equal at 32K, slower at 4K).
+ *   wave for the shapes it covers whose K tensor holds at least 192 MiB (B*L*Hkv*d*2
+ *   bytes, 1.5 x the L2 size) with B * Hkv no more than the SMs, else the single-wave
+ *   kernel (measured on one B200: the one-wave schedule is 4-6% faster with 268 MB of K,
+ *   3% slower with 134 MB, which L2 nearly holds).
  * wave = 1: the wave-scheduled kernel for every shape it covers, about 40 MB of K per
  *   wave; max_groups_per_wave > 0 caps the groups of one wave (more waves on small
  *   inputs), 0 lets the library choose.

@@ -3,15 +3,16 @@
 The wave-scheduled kernel scores the KV groups in waves (pass 1 of wave w+1 runs before
 pass 2 of wave w; each CTA merges its group's statistics after a per-wave count); the
 single-wave kernel scores every group at once.  The automatic schedule (the default)
-takes the wave-scheduled kernel with every group in one wave from 65536 tokens on, and
-the single-wave kernel below.  Every kernel and plan must give s_h and s_l within the
+takes the wave-scheduled kernel with every group in one wave when K holds at least
+192 MiB, and the single-wave kernel below.  Every kernel and plan must give s_h and s_l within the
 scoring tolerance (relative 1e-5) of the oracle on the same inputs, on shapes that cover:
 - one wave, two waves, and many waves (the two statistics slots reused);
 - a ragged last tile, the shortest eligible sequence (16 tokens, one tile), and a tile
   holding a single token;
 - 1, 2 and 4 query heads per KV head (idle epilogue warps when fewer than 4);
 - d = 64 and 128, batches of 1 to 20 sequences (160 KV groups in one launch);
-- the automatic one-wave plan at 64K+ tokens (a ragged tail, and two sequences).
+- the automatic one-wave plan with 201 and 268 MB of K (a ragged tail, and two
+  sequences).
 """
 import numpy as np
 import pytest
@@ -102,11 +103,11 @@ def test_wave_scoring_inside_a_layer_matches_the_oracle():
     _close(s_l.cpu().numpy(), ref_l, "s_l in a layer")
 
 
-@pytest.mark.parametrize("B,L,H,Hkv", [(1, 65536 + 37, 32, 8), (2, 65536, 16, 4)])
+@pytest.mark.parametrize("B,L,H,Hkv", [(1, 98304 + 37, 32, 8), (2, 65536, 32, 8)])
 def test_automatic_one_wave_schedule_matches_the_oracle(B, L, H, Hkv):
-    """From 65536 tokens on the default schedule scores every KV group in one wave of the
-    wave-scheduled kernel; it matches the oracle and the single-wave kernel, and repeated
-    launches are bit-identical."""
+    """With at least 192 MiB of K the default schedule scores every KV group in one wave
+    of the wave-scheduled kernel (here 201 and 268 MB); it matches the oracle and the
+    single-wave kernel, and repeated launches are bit-identical."""
     x = make_inputs(B, L, H, Hkv, 128, torch.bfloat16, seed=L + B)
     Q, K = x["Q"].cuda(), x["K"].cuda()
     ref_h, ref_l = oracle.score(x["Q"], x["K"], 16)

@@ -46,10 +46,11 @@ cudaError_t launch_score_wave(const tsa_dims &dm, const void *Q, const void *K, 
                               float *s_h, float *s_l, const WsLayout &w, char *ws,
                               cudaStream_t st, uint32_t limit_us, bool one_wave);
 
-// From this many tokens on, the automatic schedule scores every KV group in one wave of the
-// wave-scheduled kernel (tokens on the TMEM lanes in both passes); below it, the
-// single-wave kernel here is as fast or faster.
-constexpr int kOneWaveMinTokens = 65536;
+// From this many bytes of K on (1.5 x the L2 size), the automatic schedule scores every
+// KV group in one wave of the wave-scheduled kernel (tokens on the TMEM lanes in both
+// passes); with less K, pass 2 rereads most of K from L2 and the single-wave kernel here is
+// as fast or faster.
+constexpr double kOneWaveMinKBytes = 192.0 * (1 << 20);
 
 namespace {
 
@@ -549,7 +550,8 @@ cudaError_t launch_score_tc(const tsa_dims &dm, const void *Q, const void *K, in
                             cudaStream_t st, uint32_t limit_us, bool &fused) {
     const int mode = score_schedule();
     if (score_wave_eligible(dm, qe)) {
-        const bool one = mode == 0 && dm.L >= kOneWaveMinTokens && score_one_wave_fits(dm);
+        const double kbytes = 2.0 * dm.B * dm.L * dm.Hkv * dm.d;
+        const bool one = mode == 0 && kbytes >= kOneWaveMinKBytes && score_one_wave_fits(dm);
         if (mode == 1 || one) {
             fused = s_l != nullptr;
             return launch_score_wave(dm, Q, K, scale, s_h, s_l, w, ws, st, limit_us, one);

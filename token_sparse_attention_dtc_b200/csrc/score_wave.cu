@@ -113,7 +113,9 @@ k_score_wave(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     const int per = ntiles / S, rem = ntiles % S;
     const int first = split * per + min(split, rem), count = per + (split < rem ? 1 : 0);
     const int nphase = 2 * W;
-    unsigned int *gbar = sync, *cnt = sync + 1;  // cnt[kPartSlots]
+    // sync[0] grid barrier, sync[1..kPartSlots] per-wave counts, sync[kPartSlots + 1] the
+    // CTAs done; all zero at launch, and zero again when the last CTA is done.
+    unsigned int *gbar = sync, *cnt = sync + 1, *done = sync + 1 + kPartSlots;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -487,8 +489,8 @@ k_score_wave(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
             }
         }
         if (lane == 0) zp[((size_t)zb * nctas + cta) * kEpiWarps + ew] = zrun;
-        // Grid barrier among the epilogue warps of every CTA on gbar (zeroed before the
-        // launch), which reaches `target` = nctas times the barrier's ordinal.
+        // Grid barrier among the epilogue warps of every CTA on gbar (zero at launch),
+        // which reaches `target` = nctas times the barrier's ordinal.
         auto grid_sync = [&](unsigned target) -> bool {
             __threadfence();
             named_barrier(1, kEpiWarps * 32);
@@ -557,6 +559,17 @@ k_score_wave(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+    // Every wait of this CTA on the counters is behind it (each one either succeeded or
+    // gave up): the last CTA to get here returns them to zero for the next launch, so no
+    // memset precedes a launch.
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(done, 1u) == nctas - 1u) {
+            for (int i = 0; i < 1 + kPartSlots; ++i) atomicExch(sync + i, 0u);
+            atomicExch(done, 0u);
+            __threadfence();
+        }
     }
 }
 
@@ -635,7 +648,6 @@ static cudaError_t score_wave_impl(const tsa_dims &dm, const void *Q, const void
     uint64_t lim = (uint64_t)limit_us * 1000ull;
     int stall = test_stall();
     int L = dm.L, H = dm.H, Hkv = dm.Hkv, Bn = dm.B;
-    if ((e = cudaMemsetAsync(sync, 0, (1 + kPartSlots) * sizeof(unsigned int), st))) return e;
     void *args[] = {&tk, &tq, &L, &H, &Hkv, &Bn, &S, &gpw, &W, &sl2, (void *)&part,
                     (void *)&s_h, (void *)&s_l, (void *)&zp, (void *)&sync,
                     (void *)&ctl, &lim, &stall};
