@@ -549,6 +549,35 @@ def run_ours(args, w, L, rank, world, local_rank):
         if tsa.tsa_get_device_status(ws) != 0:
             raise RuntimeError("device error in the pages'-sparsity runs")
 
+    # the fused compress + attention + decompress (direct gather) against the staged layer,
+    # at the synthetic budget and, for long sequences, at the pages' 67.4% pruned
+    direct = None
+    if not args.no_pages_sparsity and w.dtype == torch.bfloat16:
+        direct = []
+        cases = [("synthetic budget", dict(tau=w.tau))]
+        if L >= 65536:
+            cases.append(("67.4% pruned", dict(sparsity=PAGES_SPARSITY[1])))
+        for name, kw in cases:
+            row = {"case": name}
+            for mode in (False, True):
+                for _ in range(2):
+                    tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, ws=ws, direct=mode, **kw)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                sync_all()
+                nrep = 3 if L >= 65536 else 20
+                a.record(st)
+                for _ in range(nrep):
+                    tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, ws=ws, direct=mode,
+                                  **kw)
+                b.record(st)
+                sync_all()
+                row["direct_ms" if mode else "staged_ms"] = job_max(a.elapsed_time(b) / nrep,
+                                                                    world, dev)
+            direct.append(row)
+        if tsa.tsa_get_device_status(ws) != 0:
+            raise RuntimeError("device error in the direct-gather runs")
+
     # token + block composition: block-sparse attention inside the compressed space
     blocks = None
     if not args.no_pages_sparsity and w.dtype == torch.bfloat16:  # tcgen05 path only
@@ -670,6 +699,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "graph_replay": graph,
             "pages_sparsity": pages,
             "block_sparse": blocks,
+            "direct_gather": direct,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
