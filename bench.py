@@ -898,6 +898,80 @@ def run_drift(args):
         del h, ws
 
 
+def run_kv_shard(args, w, L, rank, world, local_rank):
+    """One layer sharded by KV group over the job's ranks (token_sparse_attention_dtc_b200
+    .shard): every rank draws the same layer, keeps its KV groups' heads, and runs its part
+    (scoring of its heads, one NCCL all-gather of the partial layer scores, the rank-order
+    combination, budget, selection, gather, attention, scatter).  A step is one layer of
+    the whole job: strong scaling; the time is the max over ranks."""
+    import torch
+    import torch.distributed as dist
+
+    from token_sparse_attention_dtc_b200 import shard, tsa
+    from token_sparse_attention_dtc_b200.inputs import make_workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    tsa.lib()
+    group = None
+    if world == 1 and not dist.is_initialized():
+        import datetime
+
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29512")
+        dist.init_process_group("nccl", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=300))
+    x = make_workload(w.name, seed=args.seed, L=L, B=1)   # the same layer on every rank
+    h0, h1 = shard.head_range(w.H, w.Hkv, rank, world)
+    kv0, kv1 = shard.kv_group_range(w.Hkv, rank, world)
+    d = {"Q": x["Q"][:, :, h0:h1].contiguous().to(dev),
+         "K": x["K"][:, :, kv0:kv1].contiguous().to(dev),
+         "V": x["V"][:, :, kv0:kv1].contiguous().to(dev),
+         "X": x["X"][:, :, h0 * w.d:h1 * w.d].contiguous().to(dev)}
+    del x
+    dm = tsa.dims(d["Q"], d["K"])
+    ws = tsa.workspace(dm, w.q, device=dev)
+    Y = torch.empty_like(d["X"])
+    st = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        shard.sharded_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, group=group,
+                            ws=ws)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        a.record(st)
+        for _ in range(args.steps):
+            _, out = shard.sharded_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau,
+                                         group=group, ws=ws)
+        b.record(st)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+    ms = job_max(a.elapsed_time(b) / args.steps, world, dev)
+    if tsa.tsa_get_device_status(ws) != 0:
+        raise RuntimeError("device error in the sharded layer")
+    lk = int(out["Lkeep"].item())
+    lks = [torch.zeros(1, dtype=torch.int64, device=dev) for _ in range(world)]
+    dist.all_gather(lks, torch.tensor([lk], dtype=torch.int64, device=dev))
+    flops = 2.0 * w.H * w.d * lk * (lk + 1)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC + " (one layer sharded by KV group)", "value": ms, "unit": "ms",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": False, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": _workload_desc(w, L), "global_batch": 1, "seq_len": L,
+                       "parallelism": "kv-group shard over %d rank(s): %d query heads and "
+                                      "%d KV heads per rank (rank 0)" % (world, h1 - h0, kv1 - kv0),
+                       "exchange": "one all-gather of 4*L bytes of partial layer score per rank"},
+            "Lkeep_per_rank": [int(t.item()) for t in lks],
+            "layer_tflops": flops / (ms * 1e-3) / 1e12,
+            "clocks": clk.summary()}), flush=True)
+    if world == 1:
+        dist.destroy_process_group()
+
+
 def run_score_only(args, w, L):
     """The scoring kernel alone (tsa_score: s_h and the layer score) on the workload's Q
     and K, each launch after an L2 flush that leaves L2 clean; one JSON line with the HBM
@@ -969,6 +1043,9 @@ def main():
     ap.add_argument("--stack", action="store_true",
                     help="32-layer stack with the sparse set chosen by the drift pass")
     ap.add_argument("--sweep", action="store_true", help="tau x q sweep, B = 2, L = 64K")
+    ap.add_argument("--parallel", default="replicas", choices=("replicas", "kv"),
+                    help="N > 1: independent layers per rank (default), or one layer "
+                         "sharded by KV group across the ranks")
     ap.add_argument("--score-only", action="store_true",
                     help="time the scoring kernel alone on the workload (L2 flushed per launch)")
     ap.add_argument("--drift", action="store_true",
@@ -1012,7 +1089,10 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        run_ours(args, w, L, rank, world, local_rank)
+        if args.parallel == "kv":
+            run_kv_shard(args, w, L, rank, world, local_rank)
+        else:
+            run_ours(args, w, L, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
