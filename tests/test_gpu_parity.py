@@ -322,6 +322,27 @@ def test_layer_entry_matches_stages():
                                                     d["X"]).cpu())
 
 
+@pytest.mark.parametrize("L", [1, 129, 1000, 4096, 8192])
+def test_layer_budget_and_select_in_one_launch_match_the_oracle(L):
+    """Rows of up to 8192 tokens take budget and selection in one launch inside tsa_layer
+    (every head's CTA recomputes its batch element's budget).  L' and every index list
+    equal the oracle's on the GPU's scores, for tau = 0 (keep all), a normal tau, and a
+    tau close to 1 (keep few), with two batch elements."""
+    x = make_inputs(2, L, 8, 2, 64, torch.bfloat16, seed=L + 5)
+    d = _dev(x)
+    for tau in (0.0, 0.01, 0.999):
+        s_h = torch.empty(2, 8, L, device="cuda")
+        s_l = torch.empty(2, L, device="cuda")
+        Lk = torch.empty(2, dtype=torch.int32, device="cuda")
+        idx = torch.empty(2, 8, L, dtype=torch.int32, device="cuda")
+        tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], q=16, tau=tau, s_h=s_h, s_l=s_l,
+                      Lkeep=Lk, idx=idx)
+        lk, _ = oracle.budget(s_l.cpu().numpy(), tau)
+        np.testing.assert_array_equal(Lk.cpu().numpy(), lk, err_msg=str(tau))
+        np.testing.assert_array_equal(idx.cpu().numpy(), oracle.select(s_h.cpu().numpy(), lk),
+                                      err_msg=str(tau))
+
+
 def test_scores_are_deterministic():
     x = _dev(make_workload("llama8b_4k", seed=3))
     a = tsa.tsa_score(x["Q"], x["K"], 16)

@@ -59,6 +59,20 @@ def test_fixed_scratch_matches_tsa_score_on_consecutive_calls():
 
 
 @pytest.mark.gpu
+def test_fixed_scratch_one_wave_schedule_matches_tsa_score():
+    """At 98304 tokens of the Llama shape (201 MB of K) the scoring takes the one-wave
+    kernel, whose counters live in the fixed array too: bit for bit tsa_score's result on
+    two calls in a row."""
+    x = make_inputs(1, 98304, 32, 8, 128, torch.bfloat16, seed=13)
+    Q, K = x["Q"].cuda(), x["K"].cuda()
+    ref_h, ref_l = tsa.tsa_score(Q, K, 16)
+    for _ in range(2):
+        got_h, got_l = tsa.tsa_score_fixed_scratch(Q, K, 16)
+        assert tsa.tsa_score_fixed_scratch_status() == 0
+        assert torch.equal(got_h, ref_h) and torch.equal(got_l, ref_l)
+
+
+@pytest.mark.gpu
 def test_fixed_scratch_reports_a_device_timeout_and_recovers():
     """A bounded device wait that runs out (the stall test hook, 20 ms limit) is
     reported by tsa_score_fixed_scratch_status, once; the next call is exact again."""

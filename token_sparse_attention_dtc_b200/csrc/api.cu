@@ -535,13 +535,21 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
                             "tsa_layer pool (normalise)"));
     }
     TSA_TRY(rec(1));
-    if (o.budget == TSA_BUDGET_COVERAGE)
-        TSA_TRY(cuda_status(launch_budget(dm, s_l, o.tau, Lk, w, st), "tsa_layer budget"));
-    else
-        TSA_TRY(cuda_status(launch_fill_lkeep(dm.B, fixed_keep(dm.L, o.sparsity), Lk, st),
-                            "tsa_layer budget"));
-    TSA_TRY(rec(2));
-    TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, w, st), "tsa_layer select"));
+    if (o.budget == TSA_BUDGET_COVERAGE && budget_select_fused_fits(dm.L)) {
+        // short rows: budget and selection in one launch (both stage events after it)
+        const unsigned long long T = (unsigned long long)ceil(o.tau * 4611686018427387904.0);
+        TSA_TRY(cuda_status(launch_budget_select(dm, s_l, s_h, T, Lk, idx, (Control *)w, st),
+                            "tsa_layer budget and select"));
+        TSA_TRY(rec(2));
+    } else {
+        if (o.budget == TSA_BUDGET_COVERAGE)
+            TSA_TRY(cuda_status(launch_budget(dm, s_l, o.tau, Lk, w, st), "tsa_layer budget"));
+        else
+            TSA_TRY(cuda_status(launch_fill_lkeep(dm.B, fixed_keep(dm.L, o.sparsity), Lk, st),
+                                "tsa_layer budget"));
+        TSA_TRY(rec(2));
+        TSA_TRY(cuda_status(launch_select(dm, s_h, Lk, idx, w, st), "tsa_layer select"));
+    }
     TSA_TRY(rec(3));
     if (o.direct_gather) {  // no compressed copies: one fused attention pass
         TSA_TRY(rec(4));

@@ -97,6 +97,12 @@ cudaError_t launch_budget_cluster(const tsa_dims &dm, const float *s_l, unsigned
                                   int32_t *Lkeep, Control *ctl, cudaStream_t stream);
 cudaError_t launch_select_cluster(const tsa_dims &dm, const float *s_h, const int32_t *Lkeep,
                                   int32_t *idx, Control *ctl, cudaStream_t stream);
+// Short rows: the coverage budget and the selection in one launch (the same results as
+// launch_budget + launch_select, bit for bit).
+bool budget_select_fused_fits(int L);
+cudaError_t launch_budget_select(const tsa_dims &dm, const float *s_l, const float *s_h,
+                                 unsigned long long T, int32_t *Lkeep, int32_t *idx,
+                                 Control *ctl, cudaStream_t stream);
 
 // Host-side count of kernels this library has launched (read by tsa_kernel_launches).
 void note_launches(int n);

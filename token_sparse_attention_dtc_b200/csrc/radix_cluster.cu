@@ -35,6 +35,9 @@ constexpr int kMaxCluster = 8;          // portable cluster size
 constexpr int kBins = 4096;             // widest level
 constexpr int kRound = 4 * kThreads;    // keys per histogram round (4 per thread)
 constexpr int kCopies = 16;             // private first-level histograms (one per warp pair)
+// Rows of up to this many tokens take budget and selection in one launch, the budget
+// recomputed by every (b, h) CTA (cheaper than a second launch at these lengths).
+constexpr int kFusedMaxTokens = 8192;
 
 // Levels: bits 31..23 (sign and exponent), 22..11 and 10..0 of the key.  Scores crowd
 // into a few exponents, so the first level's atomics go to kCopies private histograms
@@ -191,6 +194,7 @@ struct BudgetShared {
     uint32_t prefix;            // digits chosen so far
     int found;                  // the last level that found its digit, plus one
     int below;                  // keys of this CTA below the threshold key
+    int keep;                   // the result, for every thread of the CTA
 };
 
 // One level of the budget search.  Returns false when the row's mass stays below T.
@@ -267,6 +271,43 @@ __device__ inline bool budget_level(const cg::cluster_group &cl, int C, uint32_t
     return S.found == LV + 1;
 }
 
+// Coverage budget of one row of layer scores, on a cluster of C CTAs that each hold one
+// slice of the row's keys: the number of tokens kept (0 when the row's mass stays below T).
+// Every CTA of the cluster returns the same value.
+__device__ inline int budget_row(const cg::cluster_group &cl, int C, uint32_t *hist0,
+                                 const uint32_t *keys, Slice sl, int L, unsigned long long T,
+                                 BudgetShared &S) {
+    const int tid = threadIdx.x;
+    if (T == 0ull) return L;  // tau = 0: nothing is pruned (no shared memory was shared yet)
+    if (tid == 0) {
+        S.prefix = 0;
+        S.before = 0;
+        S.found = 0;
+        S.below = 0;
+    }
+    // Every CTA takes the same branch: they scan the same summed histograms.
+    if (!budget_level<0>(cl, C, hist0, keys, sl.n, T, S) ||
+        !budget_level<1>(cl, C, hist0, keys, sl.n, T, S) ||
+        !budget_level<2>(cl, C, hist0, keys, sl.n, T, S)) {
+        cl.sync();  // peers may still be reading this CTA's histogram
+        return 0;   // the whole row's mass is below tau: prune everything
+    }
+    // k = (scores below the threshold key) + the copies of that key that reach tau.
+    const uint32_t P = S.prefix;
+    int below = 0;
+    for (int i = tid; i < sl.n; i += kThreads) below += keys[i] < P;
+    block_add(below, &S.below);
+    cl.sync();
+    if (tid == 0) {
+        int cnt = 0;
+        for (int c = 0; c < C; ++c) cnt += cl.map_shared_rank(&S, c)->below;
+        const unsigned long long a = mass62(P);
+        S.keep = L - (cnt + (int)((T - S.before + a - 1) / a));
+    }
+    cl.sync();  // every CTA has read every CTA's count; S.keep is visible to the CTA
+    return S.keep;
+}
+
 // grid (C, B), cluster (C, 1, 1), 1024 threads.  Dynamic shared memory: two histogram
 // buffers of 4096 (high, low) pairs of 32-bit mass-unit sums, then the slice's keys.
 __global__ void __launch_bounds__(kThreads, 1)
@@ -278,43 +319,12 @@ k_budget_cluster(const float *__restrict__ s_l, int L, int per_cta, unsigned lon
     __shared__ BudgetShared S;
     cg::cluster_group cl = cg::this_cluster();
     const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
-    const int b = blockIdx.y, tid = threadIdx.x;
+    const int b = blockIdx.y;
     const Slice sl = slice_of(cr, per_cta, L);
     if (load_keys<kLayerScoreMax>(keys, s_l + (size_t)b * L, L, sl))
         report_error(ctl, TSA_ERR_NONFINITE, 1);
-    if (T == 0ull) {  // tau = 0: nothing is pruned (no shared memory was shared yet)
-        if (cr == 0 && tid == 0) Lkeep[b] = L;
-        return;
-    }
-    if (tid == 0) {
-        S.prefix = 0;
-        S.before = 0;
-        S.found = 0;
-        S.below = 0;
-    }
-    // Every CTA takes the same branch: they scan the same summed histograms.
-    if (!budget_level<0>(cl, C, hist0, keys, sl.n, T, S) ||
-        !budget_level<1>(cl, C, hist0, keys, sl.n, T, S) ||
-        !budget_level<2>(cl, C, hist0, keys, sl.n, T, S)) {
-        // The whole row's mass is below tau: prune everything.
-        if (cr == 0 && tid == 0) Lkeep[b] = 0;
-        cl.sync();  // peers may still be reading this CTA's histogram
-        return;
-    }
-    // k = (scores below the threshold key) + the copies of that key that reach tau.
-    const uint32_t P = S.prefix;
-    int below = 0;
-    for (int i = tid; i < sl.n; i += kThreads) below += keys[i] < P;
-    block_add(below, &S.below);
-    cl.sync();
-    if (cr == 0 && tid == 0) {
-        int cnt = 0;
-        for (int c = 0; c < C; ++c) cnt += cl.map_shared_rank(&S, c)->below;
-        const unsigned long long a = mass62(P);
-        const int k = cnt + (int)((T - S.before + a - 1) / a);
-        Lkeep[b] = L - k;
-    }
-    cl.sync();  // rank 0 has read every CTA's count
+    const int keep = budget_row(cl, C, hist0, keys, sl, L, T, S);
+    if (cr == 0 && threadIdx.x == 0) Lkeep[b] = keep;
 }
 
 struct SelectShared {
@@ -383,27 +393,20 @@ __device__ inline void select_level(const cg::cluster_group &cl, int C, uint32_t
     __syncthreads();
 }
 
-// grid (C, B*H), cluster (C, 1, 1), 1024 threads.  Dynamic shared memory: two 4096-bin
-// uint32 count histograms, then the slice's keys.
-__global__ void __launch_bounds__(kThreads, 1)
-k_select_cluster(const float *__restrict__ s_h, int L, int H, int per_cta,
-                 const int32_t *__restrict__ Lkeep, int32_t *__restrict__ idx, Control *ctl) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    uint32_t *hist0 = reinterpret_cast<uint32_t *>(smem);
-    uint32_t *keys = reinterpret_cast<uint32_t *>(smem + 2 * kBins * 4);
-    __shared__ SelectShared S;
-    cg::cluster_group cl = cg::this_cluster();
-    const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
-    const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const Slice sl = slice_of(cr, per_cta, L);
-    int32_t *out = idx + (size_t)row * L;
-    const int keep = Lkeep[row / H];
+// Top-`keep` selection of one row of head scores on a cluster of C CTAs (each holding
+// one slice of the row): writes the row's index list `out`.  `keys` must have room for the
+// slice; the keys are loaded here.
+__device__ inline void select_row(const cg::cluster_group &cl, int C, int cr, uint32_t *hist0,
+                                  uint32_t *keys, Slice sl, const float *__restrict__ src,
+                                  int L, int keep, int32_t *__restrict__ out, Control *ctl,
+                                  SelectShared &S) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (keep <= 0 || keep >= L) {  // nothing or everything kept: the identity order
         for (int i = tid; i < sl.n; i += kThreads) out[sl.t0 + i] = sl.t0 + i;
         if ((keep < 0 || keep > L) && cr == 0 && tid == 0) report_error(ctl, TSA_ERR_INVALID_ARG, 2);
         return;
     }
-    if (load_keys<kHeadScoreMax>(keys, s_h + (size_t)row * L, L, sl))
+    if (load_keys<kHeadScoreMax>(keys, src, L, sl))
         report_error(ctl, TSA_ERR_NONFINITE, 3);
     if (tid == 0) {
         S.prefix = 0;
@@ -481,6 +484,49 @@ k_select_cluster(const float *__restrict__ s_h, int L, int H, int per_cta,
     cl.sync();  // peers have read this CTA's counts
 }
 
+// grid (C, B*H), cluster (C, 1, 1), 1024 threads.  Dynamic shared memory: two 4096-bin
+// uint32 count histograms, then the slice's keys.
+__global__ void __launch_bounds__(kThreads, 1)
+k_select_cluster(const float *__restrict__ s_h, int L, int H, int per_cta,
+                 const int32_t *__restrict__ Lkeep, int32_t *__restrict__ idx, Control *ctl) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *hist0 = reinterpret_cast<uint32_t *>(smem);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem + 2 * kBins * 4);
+    __shared__ SelectShared S;
+    cg::cluster_group cl = cg::this_cluster();
+    const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
+    const int row = blockIdx.y;
+    const Slice sl = slice_of(cr, per_cta, L);
+    select_row(cl, C, cr, hist0, keys, sl, s_h + (size_t)row * L, L, Lkeep[row / H],
+               idx + (size_t)row * L, ctl, S);
+}
+
+// Budget and selection in one launch for short rows (the whole row in one CTA): CTA
+// (b, h) computes batch element b's budget from s_l (every CTA of b gets the same, exact
+// integer result; head 0's CTA stores it), then selects head h's tokens with it.
+// grid (1, B*H), cluster (1, 1, 1), 1024 threads.  Dynamic shared memory: two histogram
+// buffers of 4096 (high, low) 32-bit pairs, then one row of keys (s_l's, then s_h's).
+__global__ void __launch_bounds__(kThreads, 1)
+k_budget_select(const float *__restrict__ s_l, const float *__restrict__ s_h, int L, int H,
+                unsigned long long T, int32_t *__restrict__ Lkeep, int32_t *__restrict__ idx,
+                Control *ctl) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t *hist0 = reinterpret_cast<uint32_t *>(smem);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem + 2 * kBins * 8);
+    __shared__ BudgetShared SB;
+    __shared__ SelectShared SS;
+    cg::cluster_group cl = cg::this_cluster();
+    const int row = blockIdx.y, b = row / H;
+    const Slice sl = slice_of(0, L, L);
+    if (load_keys<kLayerScoreMax>(keys, s_l + (size_t)b * L, L, sl))
+        report_error(ctl, TSA_ERR_NONFINITE, 1);
+    const int keep = budget_row(cl, 1, hist0, keys, sl, L, T, SB);
+    if (row % H == 0 && threadIdx.x == 0) Lkeep[b] = keep;
+    __syncthreads();  // the budget is done with the keys and the histograms
+    select_row(cl, 1, 0, hist0, keys, sl, s_h + (size_t)row * L, L, keep, idx + (size_t)row * L,
+               ctl, SS);
+}
+
 // Selection: the smallest cluster whose slices fit (the rows already fill the GPU).
 // Budget: one cluster per batch element, so up to 8 CTAs of at least 4096 scores each.
 // 0 when the row is too long for this path.
@@ -529,6 +575,16 @@ cudaError_t launch_budget_cluster(const tsa_dims &dm, const float *s_l, unsigned
     const int C = budget_cluster_size(dm.L), per = slice_tokens(dm.L, C);
     const size_t smem = (size_t)2 * kBins * 8 + keys_bytes(per);
     return launch_cluster(k_budget_cluster, C, dm.B, smem, stream, s_l, dm.L, per, T, Lkeep, ctl);
+}
+
+bool budget_select_fused_fits(int L) { return L <= kFusedMaxTokens; }
+
+cudaError_t launch_budget_select(const tsa_dims &dm, const float *s_l, const float *s_h,
+                                 unsigned long long T, int32_t *Lkeep, int32_t *idx,
+                                 Control *ctl, cudaStream_t stream) {
+    const size_t smem = (size_t)2 * kBins * 8 + keys_bytes(dm.L);
+    return launch_cluster(k_budget_select, 1, dm.B * dm.H, smem, stream, s_l, s_h, dm.L, dm.H,
+                          T, Lkeep, idx, ctl);
 }
 
 cudaError_t launch_select_cluster(const tsa_dims &dm, const float *s_h, const int32_t *Lkeep,
