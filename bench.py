@@ -886,6 +886,12 @@ def run_drift(args):
         ms = ev[0].elapsed_time(ev[1]) / args.steps
         nbytes = h.numel() * h.element_size()
         gbs = nbytes / (ms * 1e-3) / 1e9
+        # DRAM bytes of one launch, captured at 32 x 4096 x 4096 bf16; the bf16 walk reads
+        # every row once, so the 8192-token launch is scaled by its token count.
+        traffic = None
+        t0 = _traffic("k_drift_walk", "drift_32x4096x4096_bf16")
+        if t0 is not None and dt == torch.bfloat16 and (N, D) == (32, 4096):
+            traffic = int(t0 * T / 4096)
         print(json.dumps({
             "metric": "drift pass ms (tsa_drift: R over N layers and the delta = 0.5 mask)",
             "value": ms, "unit": "ms", "higher_is_better": False,
@@ -893,7 +899,7 @@ def run_drift(args):
             "config": {"workload": "drift: N=%d layers, T=%d tokens, d_model=%d" % (N, T, D),
                        "l2": "states %.0f MB, larger than L2; no flush" % (nbytes / 1e6)},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm"], "traffic": None,
+                         "frac": gbs / pk["hbm"], "traffic": traffic,
                          "algorithmic_bytes": nbytes}}), flush=True)
         del h, ws
 

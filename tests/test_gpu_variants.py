@@ -144,6 +144,24 @@ def test_drift_matches_oracle(dtype, T):
     _drift_check(torch.stack(h).to(dtype).contiguous(), delta=0.5)
 
 
+@pytest.mark.parametrize("dtype,N,T,D", [
+    (torch.float32, 4, 300, 4096),     # 16 KB rows: four 4 KB slices per token
+    (torch.bfloat16, 3, 70, 16384),    # 32 KB rows: eight slices
+    (torch.float32, 3, 100, 5120),     # 20 KB rows: five slices
+    (torch.bfloat16, 4, 500, 3072),    # 6 KB rows: three 2 KB slices
+    (torch.bfloat16, 2, 200, 768),     # 1.5 KB rows: three 512-byte slices
+    (torch.bfloat16, 3, 9000, 256),    # more tokens than partial slots (ragged wrap)
+    (torch.float32, 5, 4099, 96),      # 384-byte rows: the generic walk, 3 tokens past the slots
+])
+def test_drift_wide_rows_and_slot_wrap(dtype, N, T, D):
+    g = torch.Generator().manual_seed(N * T + D)
+    steps = 0.05 + torch.rand(N, generator=g) * 0.5
+    h = [torch.randn(T, D, generator=g)]
+    for l in range(N):
+        h.append(h[-1] + steps[l] * torch.randn(T, D, generator=g))
+    _drift_check(torch.stack(h).to(dtype).contiguous(), delta=0.5)
+
+
 def test_drift_identical_states_and_determinism():
     h = torch.randn(1, 300, 512).to(torch.bfloat16).expand(9, 300, 512).contiguous()
     R, mask = _drift_check(h)
