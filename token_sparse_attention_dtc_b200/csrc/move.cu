@@ -14,42 +14,58 @@ namespace tsa {
 constexpr int kMoveThreads = 256;
 constexpr int kGatherRows = 32;  // rows of one (b, h) per block
 
-// grid (B*H, ceil(L / kGatherRows)).  VPR = 16-byte vectors per row.  Heads vary
-// fastest across blocks, so the G heads that share a KV row read it close in time.
+// Rows of one (b, h) per gather block: every thread owns kQkvRows * VPR / kMoveThreads
+// vectors, and issues all their loads (index, then Q, K and V) before its first store.
+constexpr int kQkvRows = 64;
+
+// grid (B*H, ceil(L / kQkvRows)).  VPR = 16-byte vectors per row.  Heads vary fastest
+// across blocks, so the G heads that share a KV row read it close in time.
 template <int VPR>
 __global__ void __launch_bounds__(kMoveThreads)
 k_gather_qkv(const uint4 *__restrict__ Q, const uint4 *__restrict__ K, const uint4 *__restrict__ V,
              const int32_t *__restrict__ idx, const int32_t *__restrict__ Lkeep, int L, int H,
              int Hkv, uint4 *__restrict__ Qh, uint4 *__restrict__ Kh, uint4 *__restrict__ Vh,
              Control *ctl) {
+    constexpr int kPer = kQkvRows * VPR / kMoveThreads;
+    static_assert(kPer * kMoveThreads == kQkvRows * VPR, "whole vectors per thread");
     const int bh = blockIdx.x, b = bh / H, h = bh % H, kv = h / (H / Hkv);
     const int Lk = min(max(Lkeep[b], 0), L);  // a count outside [0, L] is clamped
     const int pad_end = min(L, (Lk + 127) & ~127);
-    const int i0 = blockIdx.y * kGatherRows;
+    const int i0 = blockIdx.y * kQkvRows;
     if (i0 >= pad_end) return;
     const int32_t *S = idx + (size_t)bh * L;
-    for (int e = threadIdx.x; e < kGatherRows * VPR; e += kMoveThreads) {
-        const int i = i0 + e / VPR, v = e % VPR;
-        if (i >= pad_end) break;
-        const size_t dst = ((size_t)bh * L + i) * VPR + v;
-        if (i < Lk) {
-            const int t = S[i];
-            if ((unsigned)t >= (unsigned)L) {  // not an index list of this sequence
-                report_error(ctl, TSA_ERR_INVALID_ARG, 20);
-                continue;
-            }
-            const size_t qs = (((size_t)b * L + t) * H + h) * VPR + v;
-            const size_t ks = (((size_t)b * L + t) * Hkv + kv) * VPR + v;
-            const uint4 q = Q[qs], k = K[ks], w = V[ks];
-            Qh[dst] = q;
-            Kh[dst] = k;
-            Vh[dst] = w;
+    int t[kPer];  // token of each vector's row; -1: a zero row of the padding
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int i = i0 + (threadIdx.x + u * kMoveThreads) / VPR;
+        t[u] = i < Lk ? __ldg(S + i) : -1;
+    }
+    uint4 q[kPer], k[kPer], w[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int v = (threadIdx.x + u * kMoveThreads) % VPR;
+        if ((unsigned)t[u] < (unsigned)L) {
+            const size_t qs = (((size_t)b * L + t[u]) * H + h) * VPR + v;
+            const size_t ks = (((size_t)b * L + t[u]) * Hkv + kv) * VPR + v;
+            q[u] = __ldg(Q + qs);
+            k[u] = __ldg(K + ks);
+            w[u] = __ldg(V + ks);
         } else {
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            Qh[dst] = z;
-            Kh[dst] = z;
-            Vh[dst] = z;
+            q[u] = k[u] = w[u] = make_uint4(0, 0, 0, 0);
         }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int e = threadIdx.x + u * kMoveThreads, i = i0 + e / VPR;
+        if (i >= pad_end) break;
+        if (t[u] >= L || t[u] < -1 || (t[u] == -1 && i < Lk)) {  // not an index of this sequence
+            report_error(ctl, TSA_ERR_INVALID_ARG, 20);
+            continue;
+        }
+        const size_t dst = ((size_t)bh * L + i) * VPR + e % VPR;
+        Qh[dst] = q[u];
+        Kh[dst] = k[u];
+        Vh[dst] = w[u];
     }
 }
 
@@ -154,7 +170,7 @@ cudaError_t launch_gather(const tsa_dims &dm, const void *Q, const void *K, cons
                           Control *ctl, cudaStream_t st) {
     const int esz = dm.dtype == TSA_F32 ? 4 : 2;
     const int vpr = dm.d * esz / 16;
-    dim3 grid(dm.B * dm.H, ceil_div(dm.L, kGatherRows));
+    dim3 grid(dm.B * dm.H, ceil_div(dm.L, kQkvRows));
 #define TSA_GATHER(V_)                                                                        \
     k_gather_qkv<V_><<<grid, kMoveThreads, 0, st>>>(                                         \
         (const uint4 *)Q, (const uint4 *)K, (const uint4 *)V, idx, Lkeep, dm.L, dm.H, dm.Hkv, \
