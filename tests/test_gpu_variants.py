@@ -162,6 +162,18 @@ def test_drift_wide_rows_and_slot_wrap(dtype, N, T, D):
     _drift_check(torch.stack(h).to(dtype).contiguous(), delta=0.5)
 
 
+def test_drift_bench_shape_8192_tokens():
+    """The bench's bf16 shape at 8192 tokens (two tokens per partial slot), with 4 of its 32
+    layers: the walk, the slots and the final sum are those of the timed launches."""
+    g = torch.Generator().manual_seed(8192)
+    N, T, D = 4, 8192, 4096
+    h = [torch.randn(T, D, generator=g)]
+    for l in range(N):
+        h.append(h[-1] * 0.95 + (0.1 + 0.1 * l) * torch.randn(T, D, generator=g))
+    R, mask = _drift_check(torch.stack(h).to(torch.bfloat16).contiguous())
+    assert list(mask) == [1, 1, 0, 0]
+
+
 def test_drift_identical_states_and_determinism():
     h = torch.randn(1, 300, 512).to(torch.bfloat16).expand(9, 300, 512).contiguous()
     R, mask = _drift_check(h)

@@ -135,6 +135,26 @@ __device__ inline void cluster_bins(const cg::cluster_group &cl, int C, const ui
     }
 }
 
+// Barrier over the CTAs that share histograms: the whole cluster, or this CTA alone when
+// kOne (a one-CTA launch, where a cluster barrier would only add its cost).
+template <bool kOne>
+__device__ inline void csync(const cg::cluster_group &cl) {
+    if constexpr (kOne) __syncthreads();
+    else cl.sync();
+}
+
+// cluster_bins for one CTA: plain shared-memory reads.
+template <bool kOne, int PER>
+__device__ inline void bins_of(const cg::cluster_group &cl, int C, const uint32_t *a, int d0,
+                               uint32_t (&out)[PER]) {
+    if constexpr (kOne) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) out[i] = a[d0 + i];
+    } else {
+        cluster_bins<PER>(cl, C, a, d0, out);
+    }
+}
+
 __device__ inline void zero_words(uint32_t *p, int n) {  // n a multiple of 4, p 16-byte aligned
     for (int i = threadIdx.x * 4; i < n; i += kThreads * 4)
         *reinterpret_cast<uint4 *>(p + i) = make_uint4(0, 0, 0, 0);
@@ -198,7 +218,7 @@ struct BudgetShared {
 };
 
 // One level of the budget search.  Returns false when the row's mass stays below T.
-template <int LV>
+template <int LV, bool kOne>
 __device__ inline bool budget_level(const cg::cluster_group &cl, int C, uint32_t *hist0,
                                     const uint32_t *keys, int n, unsigned long long T,
                                     BudgetShared &S) {
@@ -233,7 +253,7 @@ __device__ inline bool budget_level(const cg::cluster_group &cl, int C, uint32_t
         __syncthreads();
         fold_copies(hist0, 2 * kBins0, 2 * kBins0);
     }
-    cl.sync();  // every CTA's histogram of this level is complete
+    csync<kOne>(cl);  // every CTA's histogram of this level is complete
     // Thread t owns digits t*per .. t*per+per-1 (ascending key order).
     const int d0 = tid * per;
     unsigned long long mv[per], mine = 0;
@@ -241,8 +261,8 @@ __device__ inline bool budget_level(const cg::cluster_group &cl, int C, uint32_t
     for (int i = 0; i < per; ++i) mv[i] = 0;
     if (d0 < nb) {
         uint32_t uh[per], ul[per];
-        cluster_bins<per>(cl, C, hh, d0, uh);
-        cluster_bins<per>(cl, C, hl, d0, ul);
+        bins_of<kOne, per>(cl, C, hh, d0, uh);
+        bins_of<kOne, per>(cl, C, hl, d0, ul);
 #pragma unroll
         for (int i = 0; i < per; ++i) {
             // The bin's exponent: its own digit at the first level, else the prefix's.
@@ -274,6 +294,7 @@ __device__ inline bool budget_level(const cg::cluster_group &cl, int C, uint32_t
 // Coverage budget of one row of layer scores, on a cluster of C CTAs that each hold one
 // slice of the row's keys: the number of tokens kept (0 when the row's mass stays below T).
 // Every CTA of the cluster returns the same value.
+template <bool kOne>
 __device__ inline int budget_row(const cg::cluster_group &cl, int C, uint32_t *hist0,
                                  const uint32_t *keys, Slice sl, int L, unsigned long long T,
                                  BudgetShared &S) {
@@ -286,25 +307,27 @@ __device__ inline int budget_row(const cg::cluster_group &cl, int C, uint32_t *h
         S.below = 0;
     }
     // Every CTA takes the same branch: they scan the same summed histograms.
-    if (!budget_level<0>(cl, C, hist0, keys, sl.n, T, S) ||
-        !budget_level<1>(cl, C, hist0, keys, sl.n, T, S) ||
-        !budget_level<2>(cl, C, hist0, keys, sl.n, T, S)) {
-        cl.sync();  // peers may still be reading this CTA's histogram
-        return 0;   // the whole row's mass is below tau: prune everything
+    if (!budget_level<0, kOne>(cl, C, hist0, keys, sl.n, T, S) ||
+        !budget_level<1, kOne>(cl, C, hist0, keys, sl.n, T, S) ||
+        !budget_level<2, kOne>(cl, C, hist0, keys, sl.n, T, S)) {
+        csync<kOne>(cl);  // peers may still be reading this CTA's histogram
+        return 0;         // the whole row's mass is below tau: prune everything
     }
     // k = (scores below the threshold key) + the copies of that key that reach tau.
     const uint32_t P = S.prefix;
     int below = 0;
     for (int i = tid; i < sl.n; i += kThreads) below += keys[i] < P;
     block_add(below, &S.below);
-    cl.sync();
+    csync<kOne>(cl);
     if (tid == 0) {
         int cnt = 0;
-        for (int c = 0; c < C; ++c) cnt += cl.map_shared_rank(&S, c)->below;
+        if constexpr (kOne) cnt = S.below;
+        else
+            for (int c = 0; c < C; ++c) cnt += cl.map_shared_rank(&S, c)->below;
         const unsigned long long a = mass62(P);
         S.keep = L - (cnt + (int)((T - S.before + a - 1) / a));
     }
-    cl.sync();  // every CTA has read every CTA's count; S.keep is visible to the CTA
+    csync<kOne>(cl);  // every CTA has read every CTA's count; S.keep is visible to the CTA
     return S.keep;
 }
 
@@ -323,7 +346,7 @@ k_budget_cluster(const float *__restrict__ s_l, int L, int per_cta, unsigned lon
     const Slice sl = slice_of(cr, per_cta, L);
     if (load_keys<kLayerScoreMax>(keys, s_l + (size_t)b * L, L, sl))
         report_error(ctl, TSA_ERR_NONFINITE, 1);
-    const int keep = budget_row(cl, C, hist0, keys, sl, L, T, S);
+    const int keep = budget_row<false>(cl, C, hist0, keys, sl, L, T, S);
     if (cr == 0 && threadIdx.x == 0) Lkeep[b] = keep;
 }
 
@@ -337,7 +360,7 @@ struct SelectShared {
 };
 
 // One level of the top-k search: narrows S.prefix and S.need.
-template <int LV>
+template <int LV, bool kOne>
 __device__ inline void select_level(const cg::cluster_group &cl, int C, uint32_t *hist0,
                                     const uint32_t *keys, int n, SelectShared &S) {
     constexpr int shift = lv_shift(LV), nb = 1 << lv_bits(LV);
@@ -363,13 +386,13 @@ __device__ inline void select_level(const cg::cluster_group &cl, int C, uint32_t
         __syncthreads();
         fold_copies(hist0, kBins0, kBins0);
     }
-    cl.sync();
+    csync<kOne>(cl);
     // Thread t sums digits t*per .. t*per+per-1; threads past the digits own none.
     const int d0 = tid * per;
     uint32_t cnt[per];
 #pragma unroll
     for (int i = 0; i < per; ++i) cnt[i] = 0;
-    if (d0 < nb) cluster_bins<per>(cl, C, h, d0, cnt);
+    if (d0 < nb) bins_of<kOne, per>(cl, C, h, d0, cnt);
     int mine = 0;
 #pragma unroll
     for (int i = 0; i < per; ++i) mine += (int)cnt[i];
@@ -396,6 +419,7 @@ __device__ inline void select_level(const cg::cluster_group &cl, int C, uint32_t
 // Top-`keep` selection of one row of head scores on a cluster of C CTAs (each holding
 // one slice of the row): writes the row's index list `out`.  `keys` must have room for the
 // slice; the keys are loaded here.
+template <bool kOne>
 __device__ inline void select_row(const cg::cluster_group &cl, int C, int cr, uint32_t *hist0,
                                   uint32_t *keys, Slice sl, const float *__restrict__ src,
                                   int L, int keep, int32_t *__restrict__ out, Control *ctl,
@@ -412,9 +436,9 @@ __device__ inline void select_row(const cg::cluster_group &cl, int C, int cr, ui
         S.prefix = 0;
         S.need = keep;
     }
-    select_level<0>(cl, C, hist0, keys, sl.n, S);
-    select_level<1>(cl, C, hist0, keys, sl.n, S);
-    select_level<2>(cl, C, hist0, keys, sl.n, S);
+    select_level<0, kOne>(cl, C, hist0, keys, sl.n, S);
+    select_level<1, kOne>(cl, C, hist0, keys, sl.n, S);
+    select_level<2, kOne>(cl, C, hist0, keys, sl.n, S);
     // Threshold key P; the first `take` keys equal to P (in token order) are kept.
     const uint32_t P = S.prefix;
     const int take = S.need;
@@ -443,7 +467,7 @@ __device__ inline void select_row(const cg::cluster_group &cl, int C, int cr, ui
             S.eq = e;
         }
     }
-    cl.sync();  // every CTA's counts are final
+    csync<kOne>(cl);  // every CTA's counts are final
     if (tid == 0) {
         int eq_before = 0, sel_base = 0;
         for (int c = 0; c < cr; ++c) {
@@ -481,7 +505,7 @@ __device__ inline void select_row(const cg::cluster_group &cl, int C, int cr, ui
         selb += __popc(sm);
         restb += __popc(rm);
     }
-    cl.sync();  // peers have read this CTA's counts
+    csync<kOne>(cl);  // peers have read this CTA's counts
 }
 
 // grid (C, B*H), cluster (C, 1, 1), 1024 threads.  Dynamic shared memory: two 4096-bin
@@ -497,8 +521,8 @@ k_select_cluster(const float *__restrict__ s_h, int L, int H, int per_cta,
     const int C = (int)cl.num_blocks(), cr = (int)cl.block_rank();
     const int row = blockIdx.y;
     const Slice sl = slice_of(cr, per_cta, L);
-    select_row(cl, C, cr, hist0, keys, sl, s_h + (size_t)row * L, L, Lkeep[row / H],
-               idx + (size_t)row * L, ctl, S);
+    select_row<false>(cl, C, cr, hist0, keys, sl, s_h + (size_t)row * L, L, Lkeep[row / H],
+                      idx + (size_t)row * L, ctl, S);
 }
 
 // Budget and selection in one launch for short rows (the whole row in one CTA): CTA
@@ -520,11 +544,11 @@ k_budget_select(const float *__restrict__ s_l, const float *__restrict__ s_h, in
     const Slice sl = slice_of(0, L, L);
     if (load_keys<kLayerScoreMax>(keys, s_l + (size_t)b * L, L, sl))
         report_error(ctl, TSA_ERR_NONFINITE, 1);
-    const int keep = budget_row(cl, 1, hist0, keys, sl, L, T, SB);
+    const int keep = budget_row<true>(cl, 1, hist0, keys, sl, L, T, SB);
     if (row % H == 0 && threadIdx.x == 0) Lkeep[b] = keep;
     __syncthreads();  // the budget is done with the keys and the histograms
-    select_row(cl, 1, 0, hist0, keys, sl, s_h + (size_t)row * L, L, keep, idx + (size_t)row * L,
-               ctl, SS);
+    select_row<true>(cl, 1, 0, hist0, keys, sl, s_h + (size_t)row * L, L, keep,
+                     idx + (size_t)row * L, ctl, SS);
 }
 
 // Selection: the smallest cluster whose slices fit (the rows already fill the GPU).
