@@ -379,12 +379,23 @@ def run_ours(args, w, L, rank, world, local_rank):
         t_start.record(st)
         for s in range(args.steps):
             tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk,
-                          idx=idx, ws=ws, stage_events=evs[s])
+                          idx=idx, ws=ws)
         t_stop.record(st)
         n_launches = tsa.kernel_launches() - n_launch0
         sync_all()
     total_ms = t_start.elapsed_time(t_stop)
     ms_step = total_ms / args.steps
+    # The stage breakdown: the same steps again, with an event between every two stages
+    # (the events hold each kernel back until the one before it has finished, so this
+    # loop's layer time is reported on its own).
+    sync_all()
+    t_start.record(st)
+    for s in range(args.steps):
+        tsa.tsa_layer(d["Q"], d["K"], d["V"], d["X"], Y, q=w.q, tau=w.tau, Lkeep=Lk,
+                      idx=idx, ws=ws, stage_events=evs[s])
+    t_stop.record(st)
+    sync_all()
+    ms_step_staged = job_max(t_start.elapsed_time(t_stop) / args.steps, world, dev)
     stage_ms = {name: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1])
                                       for s in range(args.steps))
                 for i, name in enumerate(STAGES)}
@@ -691,6 +702,7 @@ def run_ours(args, w, L, rank, world, local_rank):
                        "Lkeep": lk, "kept_fraction": lk / L},
             "roofline": roof,
             "stages_ms": stage_ms,
+            "layer_ms_with_stage_events": ms_step_staged,
             "hbm_kernels": hbm_roof,
             "attn_tflops": attn_tf,
             "layer_tflops": flops / (ms_step * 1e-3) / 1e12,

@@ -39,14 +39,14 @@ cudaError_t launch_select(const tsa_dims &, const float *, const int32_t *, int3
                           cudaStream_t);
 cudaError_t launch_gather(const tsa_dims &, const void *, const void *, const void *,
                           const int32_t *, const int32_t *, void *, void *, void *, Control *,
-                          cudaStream_t);
+                          cudaStream_t, bool = false);
 cudaError_t launch_attn_simt(const tsa_dims &, const void *, const void *, const void *,
                              const int32_t *, int, float, void *, cudaStream_t);
 cudaError_t launch_attn_tc(const tsa_dims &, const void *, const void *, const void *,
                            const int32_t *, int, float, void *, Control *, cudaStream_t,
-                           uint32_t, const uint32_t * = nullptr);
+                           uint32_t, const uint32_t * = nullptr, bool = false);
 cudaError_t launch_scatter(const tsa_dims &, const void *, const int32_t *, const int32_t *,
-                           const void *, void *, cudaStream_t);
+                           const void *, void *, cudaStream_t, bool = false);
 cudaError_t launch_head_sum(const tsa_dims &, const float *, float *, cudaStream_t);
 cudaError_t launch_combine_parts(int, int, int, const float *, float *, float *, cudaStream_t);
 
@@ -199,11 +199,11 @@ static tsa_status do_score(const tsa_dims &dm, const void *Q, const void *K, int
 
 static tsa_status do_attn(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                           const int32_t *Lkeep, int dense, float scale, void *O, char *ws,
-                          cudaStream_t st, const uint32_t *bmask = nullptr) {
+                          cudaStream_t st, const uint32_t *bmask = nullptr, bool pdl = false) {
     cudaError_t e;
     if (dm.dtype == TSA_BF16)
         e = launch_attn_tc(dm, Q, K, V, Lkeep, dense, scale, O, reinterpret_cast<Control *>(ws),
-                           st, g_wait_limit_us, bmask);
+                           st, g_wait_limit_us, bmask, pdl);
     else
         e = launch_attn_simt(dm, Q, K, V, Lkeep, dense, scale, O, st);
     return cuda_status(e, "tsa_attn");
@@ -512,6 +512,10 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
         return cuda_status(cudaEventRecord((cudaEvent_t)stage_events[i], st), "event record");
     };
     const bool pooled = o.pool != TSA_POOL_NONE;
+    // The kernels after the scoring are launched as a programmatic-dependent chain (each
+    // may launch while the one before it finishes, and waits for it before reading its
+    // results) unless stage events are recorded between them.
+    const bool pdl = !stage_events;
     // Scores used by budget and selection: the raw ones, or the pooled ones.
     float *s_raw = (s_h_out && !pooled) ? s_h_out : (float *)(w + y.s_h);
     float *s_h = !pooled ? s_raw : (s_h_out ? s_h_out : (float *)(w + y.s_hp));
@@ -538,7 +542,8 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
     if (o.budget == TSA_BUDGET_COVERAGE && budget_select_fused_fits(dm.L)) {
         // short rows: budget and selection in one launch (both stage events after it)
         const unsigned long long T = (unsigned long long)ceil(o.tau * 4611686018427387904.0);
-        TSA_TRY(cuda_status(launch_budget_select(dm, s_l, s_h, T, Lk, idx, (Control *)w, st),
+        TSA_TRY(cuda_status(launch_budget_select(dm, s_l, s_h, T, Lk, idx, (Control *)w, st,
+                                                 pdl && !pooled),
                             "tsa_layer budget and select"));
         TSA_TRY(rec(2));
     } else {
@@ -557,7 +562,7 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
         TSA_TRY(rec(5));
         return rec(6);
     }
-    TSA_TRY(cuda_status(launch_gather(dm, Q, K, V, idx, Lk, Qh, Kh, Vh, (Control *)w, st),
+    TSA_TRY(cuda_status(launch_gather(dm, Q, K, V, idx, Lk, Qh, Kh, Vh, (Control *)w, st, pdl),
                         "tsa_layer gather"));
     TSA_TRY(rec(4));
     uint32_t *bm = nullptr;
@@ -567,9 +572,9 @@ static tsa_status layer_impl(const tsa_dims *dims, const void *Q, const void *K,
                                                 nullptr, bm, w + y.blk_scratch, st),
                             "tsa_layer block select"));
     }
-    TSA_TRY(do_attn(dm, Qh, Kh, Vh, Lk, 0, scale, Oh, w, st, bm));
+    TSA_TRY(do_attn(dm, Qh, Kh, Vh, Lk, 0, scale, Oh, w, st, bm, pdl && !blocks));
     TSA_TRY(rec(5));
-    TSA_TRY(cuda_status(launch_scatter(dm, Oh, idx, Lk, X, Y, st), "tsa_layer scatter"));
+    TSA_TRY(cuda_status(launch_scatter(dm, Oh, idx, Lk, X, Y, st, pdl), "tsa_layer scatter"));
     return rec(6);
 }
 

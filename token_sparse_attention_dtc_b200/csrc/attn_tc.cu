@@ -256,6 +256,8 @@ k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
     // CTA order: groups of `hgroup` heads whose K/V fit in L2 together, one group after
     // the other; inside a group the heaviest pairs of all its heads come first.  The CTAs in
     // flight share their heads' K/V tiles in L2, and the light pairs fill the tail.
+    pdl_wait();  // Q, K, V and the kept counts are the previous kernels'
+    pdl_trigger();
     const int npairs = ceil_div(L, 2 * kBM), B_H = gridDim.x / npairs;
     const int grp = blockIdx.x / (hgroup * npairs), r = blockIdx.x % (hgroup * npairs);
     const int ghead = min(hgroup, B_H - grp * hgroup);  // heads in this group
@@ -527,7 +529,7 @@ template <int D, bool kGather>
 static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                                 const int32_t *Lkeep, int dense, float scale, void *O,
                                 const GatherArgs &ga, const uint32_t *bmask, Control *ctl,
-                                cudaStream_t st, uint32_t limit_us) {
+                                cudaStream_t st, uint32_t limit_us, bool pdl = false) {
     CUtensorMap tq, tk, tv;
     memset(&tq, 0, sizeof tq);  // the direct-gather mode reads no tensor map
     memset(&tk, 0, sizeof tk);
@@ -560,21 +562,22 @@ static cudaError_t attn_tc_impl(const tsa_dims &dm, const void *Q, const void *K
     constexpr size_t kL2Share = 64u << 20;
     const size_t kv_head = (size_t)4 * dm.L * D;
     const int hgroup = (int)std::max<size_t>(1, std::min<size_t>((size_t)dm.B * dm.H, kL2Share / kv_head));
-    k_attn_tc<D, kGather><<<(unsigned)nblocks, kGather ? kGatherThreads : kThreads, smem, st>>>(
-        tq, tk, tv, Lkeep, dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f,
-        (__nv_bfloat16 *)O, ga, bmask, hgroup, ctl, (uint64_t)limit_us * 1000ull, test_stall());
+    e = launch_k(k_attn_tc<D, kGather>, dim3((unsigned)nblocks),
+                 dim3(kGather ? kGatherThreads : kThreads), smem, st, pdl, tq, tk, tv, Lkeep,
+                 dense, dm.L, dm.H, dm.Hkv, scale * 1.4426950408889634f, (__nv_bfloat16 *)O, ga,
+                 bmask, hgroup, ctl, (uint64_t)limit_us * 1000ull, test_stall());
     note_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_attn_tc(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                            const int32_t *Lkeep, int dense, float scale, void *O, Control *ctl,
-                           cudaStream_t st, uint32_t limit_us, const uint32_t *bmask) {
+                           cudaStream_t st, uint32_t limit_us, const uint32_t *bmask, bool pdl) {
     const GatherArgs none{};
     return dm.d == 64 ? attn_tc_impl<64, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, bmask,
-                                                ctl, st, limit_us)
+                                                ctl, st, limit_us, pdl)
                       : attn_tc_impl<128, false>(dm, Q, K, V, Lkeep, dense, scale, O, none, bmask,
-                                                 ctl, st, limit_us);
+                                                 ctl, st, limit_us, pdl);
 }
 
 // Compressed attention reading Q, K, V rows through idx, with Y = X + Ô written into the

@@ -27,6 +27,37 @@ inline size_t score_wave_bytes(int B) { return kScoreWavePartBytes + size_t(B) *
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the kernel before it in the stream is still running:
+// pdl_wait() returns once that kernel has completed and its writes are visible, and
+// pdl_trigger() lets the next such kernel start launching.  Kernels call pdl_trigger()
+// only after pdl_wait(), so every kernel of a chain sees the writes of all the kernels
+// before it.  Both are no-ops in a kernel launched the ordinary way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch of `k` on `st`; with pdl, the launch may overlap the tail of the kernel before it
+// (the kernel must begin with pdl_wait()).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t st, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    if (pdl) {
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
+
 // Device error reporting: the first error wins.
 __device__ inline void report_error(Control *c, int code, int where) {
     if (atomicCAS(&c->err, 0, code) == 0) c->err_where = where;
@@ -102,7 +133,7 @@ cudaError_t launch_select_cluster(const tsa_dims &dm, const float *s_h, const in
 bool budget_select_fused_fits(int L);
 cudaError_t launch_budget_select(const tsa_dims &dm, const float *s_l, const float *s_h,
                                  unsigned long long T, int32_t *Lkeep, int32_t *idx,
-                                 Control *ctl, cudaStream_t stream);
+                                 Control *ctl, cudaStream_t stream, bool pdl = false);
 
 // Host-side count of kernels this library has launched (read by tsa_kernel_launches).
 void note_launches(int n);

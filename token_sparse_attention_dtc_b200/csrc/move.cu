@@ -28,6 +28,8 @@ k_gather_qkv(const uint4 *__restrict__ Q, const uint4 *__restrict__ K, const uin
              Control *ctl) {
     constexpr int kPer = kQkvRows * VPR / kMoveThreads;
     static_assert(kPer * kMoveThreads == kQkvRows * VPR, "whole vectors per thread");
+    pdl_wait();  // the index lists and counts are the previous kernels'
+    pdl_trigger();
     const int bh = blockIdx.x, b = bh / H, h = bh % H, kv = h / (H / Hkv);
     const int Lk = min(max(Lkeep[b], 0), L);  // a count outside [0, L] is clamped
     const int pad_end = min(L, (Lk + 127) & ~127);
@@ -119,6 +121,8 @@ template <typename T, int VPR, bool in_place>
 __global__ void __launch_bounds__(kMoveThreads)
 k_scatter_residual(const uint4 *__restrict__ Oh, const int32_t *__restrict__ idx,
                    const int32_t *__restrict__ Lkeep, const uint4 *X, uint4 *Y, int L, int H) {
+    pdl_wait();  // Ô is the previous kernel's
+    pdl_trigger();
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int Lk = min(max(Lkeep[b], 0), L);  // a count outside [0, L] is clamped
     const int i0 = blockIdx.y * kGatherRows;
@@ -167,14 +171,15 @@ k_residual_dense(const uint4 *__restrict__ O, const uint4 *X, uint4 *Y, size_t n
 
 cudaError_t launch_gather(const tsa_dims &dm, const void *Q, const void *K, const void *V,
                           const int32_t *idx, const int32_t *Lkeep, void *Qh, void *Kh, void *Vh,
-                          Control *ctl, cudaStream_t st) {
+                          Control *ctl, cudaStream_t st, bool pdl) {
     const int esz = dm.dtype == TSA_F32 ? 4 : 2;
     const int vpr = dm.d * esz / 16;
     dim3 grid(dm.B * dm.H, ceil_div(dm.L, kQkvRows));
-#define TSA_GATHER(V_)                                                                        \
-    k_gather_qkv<V_><<<grid, kMoveThreads, 0, st>>>(                                         \
-        (const uint4 *)Q, (const uint4 *)K, (const uint4 *)V, idx, Lkeep, dm.L, dm.H, dm.Hkv, \
-        (uint4 *)Qh, (uint4 *)Kh, (uint4 *)Vh, ctl)
+    cudaError_t e;
+#define TSA_GATHER(V_)                                                                       \
+    e = launch_k(k_gather_qkv<V_>, grid, dim3(kMoveThreads), 0, st, pdl, (const uint4 *)Q,  \
+                 (const uint4 *)K, (const uint4 *)V, idx, Lkeep, dm.L, dm.H, dm.Hkv,          \
+                 (uint4 *)Qh, (uint4 *)Kh, (uint4 *)Vh, ctl)
     switch (vpr) {
         case 8: TSA_GATHER(8); break;
         case 16: TSA_GATHER(16); break;
@@ -183,12 +188,13 @@ cudaError_t launch_gather(const tsa_dims &dm, const void *Q, const void *K, cons
     }
 #undef TSA_GATHER
     note_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 template <typename T>
 static cudaError_t scatter_impl(const tsa_dims &dm, const void *Oh, const int32_t *idx,
-                                const int32_t *Lkeep, const void *X, void *Y, cudaStream_t st) {
+                                const int32_t *Lkeep, const void *X, void *Y, cudaStream_t st,
+                                bool pdl) {
     const int vpr = dm.d * (int)sizeof(T) / 16;
     if (!idx) {
         const size_t nvec = (size_t)dm.B * dm.L * dm.H * vpr;
@@ -201,13 +207,14 @@ static cudaError_t scatter_impl(const tsa_dims &dm, const void *Oh, const int32_
     }
     dim3 grid(dm.B * dm.H, ceil_div(dm.L, kGatherRows));
     const bool ip = (X == Y);
+    cudaError_t e;
 #define TSA_SCATTER(V_)                                                                     \
-    if (ip)                                                                                 \
-        k_scatter_residual<T, V_, true><<<grid, kMoveThreads, 0, st>>>(                     \
-            (const uint4 *)Oh, idx, Lkeep, (const uint4 *)X, (uint4 *)Y, dm.L, dm.H);       \
-    else                                                                                    \
-        k_scatter_residual<T, V_, false><<<grid, kMoveThreads, 0, st>>>(                    \
-            (const uint4 *)Oh, idx, Lkeep, (const uint4 *)X, (uint4 *)Y, dm.L, dm.H)
+    e = ip ? launch_k(k_scatter_residual<T, V_, true>, grid, dim3(kMoveThreads), 0, st, pdl, \
+                      (const uint4 *)Oh, idx, Lkeep, (const uint4 *)X, (uint4 *)Y, dm.L,     \
+                      dm.H)                                                                  \
+           : launch_k(k_scatter_residual<T, V_, false>, grid, dim3(kMoveThreads), 0, st,     \
+                      pdl, (const uint4 *)Oh, idx, Lkeep, (const uint4 *)X, (uint4 *)Y,      \
+                      dm.L, dm.H)
     switch (vpr) {
         case 8: TSA_SCATTER(8); break;
         case 16: TSA_SCATTER(16); break;
@@ -216,13 +223,14 @@ static cudaError_t scatter_impl(const tsa_dims &dm, const void *Oh, const int32_
     }
 #undef TSA_SCATTER
     note_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_scatter(const tsa_dims &dm, const void *Oh, const int32_t *idx,
-                           const int32_t *Lkeep, const void *X, void *Y, cudaStream_t st) {
-    return dm.dtype == TSA_F32 ? scatter_impl<float>(dm, Oh, idx, Lkeep, X, Y, st)
-                               : scatter_impl<__nv_bfloat16>(dm, Oh, idx, Lkeep, X, Y, st);
+                           const int32_t *Lkeep, const void *X, void *Y, cudaStream_t st,
+                           bool pdl) {
+    return dm.dtype == TSA_F32 ? scatter_impl<float>(dm, Oh, idx, Lkeep, X, Y, st, pdl)
+                               : scatter_impl<__nv_bfloat16>(dm, Oh, idx, Lkeep, X, Y, st, pdl);
 }
 
 cudaError_t launch_copy_rest(const tsa_dims &dm, const int32_t *idx, const int32_t *Lkeep,

@@ -541,6 +541,8 @@ k_budget_select(const float *__restrict__ s_l, const float *__restrict__ s_h, in
     __shared__ SelectShared SS;
     cg::cluster_group cl = cg::this_cluster();
     const int row = blockIdx.y, b = row / H;
+    pdl_wait();  // the scores are the previous kernel's
+    pdl_trigger();
     const Slice sl = slice_of(0, L, L);
     if (load_keys<kLayerScoreMax>(keys, s_l + (size_t)b * L, L, sl))
         report_error(ctl, TSA_ERR_NONFINITE, 1);
@@ -570,7 +572,7 @@ int slice_tokens(int L, int C) { return (ceil_div(L, C) + 3) & ~3; }
 size_t keys_bytes(int per_cta) { return (size_t)4 * ceil_div(per_cta, kRound) * kRound; }
 
 template <typename Kernel, typename... Args>
-cudaError_t launch_cluster(Kernel k, int C, int rows, size_t smem, cudaStream_t stream,
+cudaError_t launch_cluster(Kernel k, int C, int rows, size_t smem, cudaStream_t stream, bool pdl,
                            Args... args) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -579,13 +581,15 @@ cudaError_t launch_cluster(Kernel k, int C, int rows, size_t smem, cudaStream_t 
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = C;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 2 : 1;
     note_launches(1);
     return cudaLaunchKernelEx(&cfg, k, args...);
 }
@@ -598,25 +602,26 @@ cudaError_t launch_budget_cluster(const tsa_dims &dm, const float *s_l, unsigned
                                   int32_t *Lkeep, Control *ctl, cudaStream_t stream) {
     const int C = budget_cluster_size(dm.L), per = slice_tokens(dm.L, C);
     const size_t smem = (size_t)2 * kBins * 8 + keys_bytes(per);
-    return launch_cluster(k_budget_cluster, C, dm.B, smem, stream, s_l, dm.L, per, T, Lkeep, ctl);
+    return launch_cluster(k_budget_cluster, C, dm.B, smem, stream, false, s_l, dm.L, per, T, Lkeep,
+                          ctl);
 }
 
 bool budget_select_fused_fits(int L) { return L <= kFusedMaxTokens; }
 
 cudaError_t launch_budget_select(const tsa_dims &dm, const float *s_l, const float *s_h,
                                  unsigned long long T, int32_t *Lkeep, int32_t *idx,
-                                 Control *ctl, cudaStream_t stream) {
+                                 Control *ctl, cudaStream_t stream, bool pdl) {
     const size_t smem = (size_t)2 * kBins * 8 + keys_bytes(dm.L);
-    return launch_cluster(k_budget_select, 1, dm.B * dm.H, smem, stream, s_l, s_h, dm.L, dm.H,
-                          T, Lkeep, idx, ctl);
+    return launch_cluster(k_budget_select, 1, dm.B * dm.H, smem, stream, pdl, s_l, s_h, dm.L,
+                          dm.H, T, Lkeep, idx, ctl);
 }
 
 cudaError_t launch_select_cluster(const tsa_dims &dm, const float *s_h, const int32_t *Lkeep,
                                   int32_t *idx, Control *ctl, cudaStream_t stream) {
     const int C = cluster_size(dm.L), per = slice_tokens(dm.L, C);
     const size_t smem = (size_t)2 * kBins * 4 + keys_bytes(per);
-    return launch_cluster(k_select_cluster, C, dm.B * dm.H, smem, stream, s_h, dm.L, dm.H, per,
-                          Lkeep, idx, ctl);
+    return launch_cluster(k_select_cluster, C, dm.B * dm.H, smem, stream, false, s_h, dm.L, dm.H,
+                          per, Lkeep, idx, ctl);
 }
 
 }  // namespace tsa

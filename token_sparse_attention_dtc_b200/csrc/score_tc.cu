@@ -112,6 +112,9 @@ k_score_tc(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16 *__restr
            int H, int Hkv, int qe, float sl2, int nsplit, int group0, float2 *part,
            float *__restrict__ s_h, float *__restrict__ s_l, float *__restrict__ norm_part,
            unsigned int *gbar, Control *ctl, uint64_t limit_ns, int stall) {
+    // The kernel after this one in a layer (budget and selection) may start launching; it
+    // waits for this grid to complete before it reads the scores.
+    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     ScoreSmem<D> &sm = *reinterpret_cast<ScoreSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

@@ -102,6 +102,9 @@ k_score_wave(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CU
              int L, int H, int Hkv, int Bn, int S, int gpw, int W, float sl2, float2 *part,
              float *__restrict__ s_h, float *__restrict__ s_l, float *zp, unsigned int *sync,
              Control *ctl, uint64_t limit_ns, int stall) {
+    // The kernel after this one in a layer (budget and selection) may start launching; it
+    // waits for this grid to complete before it reads the scores.
+    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     WaveSmem<D> &sm = *reinterpret_cast<WaveSmem<D> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
