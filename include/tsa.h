@@ -198,7 +198,10 @@ TSA_API tsa_status tsa_scatter_residual(const tsa_dims *dims, const void *Oh, co
  * points to 7 cudaEvent_t (as void*) recorded before scoring and after each of the
  * six stages (for a dense layer the first five are recorded at the start; for L <= 8192
  * budget and selection run in one launch, and the events after them are recorded
- * together).  Y may equal X. */
+ * together).  Without stage events the kernels after the scoring are launched as a
+ * programmatic-dependent chain (each may start launching while the one before it
+ * finishes; the results are the same bit for bit); with them, each kernel waits for the
+ * event before it.  Y may equal X. */
 TSA_API tsa_status tsa_layer(const tsa_dims *dims, const void *Q, const void *K, const void *V,
                      const void *X, void *Y, int32_t is_sparse, int32_t q, double tau,
                      float scale, float *s_h_out, float *s_l_out, int32_t *Lkeep_out,
