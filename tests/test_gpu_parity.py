@@ -322,6 +322,31 @@ def test_layer_entry_matches_stages():
                                                     d["X"]).cpu())
 
 
+@pytest.mark.parametrize("wl,L", [("llama8b_4k", None), ("llama8b_32k", 16384)])
+def test_layer_launch_chain_with_and_without_stage_events(wl, L):
+    """Without stage events tsa_layer launches the kernels after the scoring as a
+    programmatic-dependent chain; with them, each waits for its event.  Both give the same
+    layer bit for bit, layer after layer in place (each layer reads the Y the one before
+    wrote), also through the grid-wide budget and selection of rows over 8192 tokens."""
+    x = make_workload(wl, seed=4, L=L)
+    d = _dev(x)
+    outs = []
+    for use_events in (False, True):
+        Y = d["X"].clone()
+        Lk = torch.empty(1, dtype=torch.int32, device="cuda")
+        idx = torch.empty(1, 32, Y.shape[1], dtype=torch.int32, device="cuda")
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(7)] if use_events else None
+        for e in ev or []:
+            e.record()  # creates the event (torch makes it on first use)
+        for _ in range(3):
+            tsa.tsa_layer(d["Q"], d["K"], d["V"], Y, Y, q=16, tau=0.01, Lkeep=Lk, idx=idx,
+                          stage_events=ev)
+        torch.cuda.synchronize()
+        outs.append((Y.cpu(), Lk.cpu(), idx.cpu()))
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+
+
 @pytest.mark.parametrize("L", [1, 129, 1000, 4096, 8192])
 def test_layer_budget_and_select_in_one_launch_match_the_oracle(L):
     """Rows of up to 8192 tokens take budget and selection in one launch inside tsa_layer
