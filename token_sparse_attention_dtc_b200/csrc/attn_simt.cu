@@ -1,12 +1,15 @@
 // Causal attention on CUDA cores for fp32 inputs (the fp32 path keeps full fp32
 // products; tensor-core tf32 would not meet a 1e-4 output tolerance).  bf16 inputs run on
 // the tensor cores (attn_tc.cu).  Flash-style
-// online softmax over 64-key tiles, one block per (64-row query tile, batch, head).
+// online softmax over 64-key tiles, one block per (32-row query tile, batch, head).
 //
 // Method: "Token Sparse Attention" papernotes.org notes, 整体框架 (dense attention on
 // the compressed L'×L' problem); bxzpzcl.cn post §1.1 (softmax(Q̂K̂ᵀ/√d)V̂).  The causal
 // mask j <= i in compressed order equals the mask on original positions because the
 // index lists are ascending.
+//
+// 32-row query tiles (8 threads per row, each 8 key columns of S and D/8 output columns),
+// so that short rows still spread over many blocks.
 #include <math.h>
 
 #include "common.cuh"
@@ -14,7 +17,9 @@
 namespace tsa {
 
 constexpr int kAttnSimtThreads = 256;
-constexpr int kBM = 64, kBN = 64;
+constexpr int kBM = 32, kBN = 64;
+constexpr int kTPR = kAttnSimtThreads / kBM;  // threads per query row
+constexpr int kSC = kBN / kTPR;               // key columns of S per thread
 
 template <int D> struct SimtSmem {
     float q[kBM][D + 1];
@@ -48,8 +53,8 @@ k_attn_simt(const T *__restrict__ Q, const T *__restrict__ K, const T *__restric
         qbase = kbase = (size_t)bh * L * D;
         qstride = kstride = D;
     }
-    const int tid = threadIdx.x, r = tid >> 2, cg = tid & 3;
-    constexpr int OC = D / 4;  // output columns per thread
+    const int tid = threadIdx.x, r = tid / kTPR, cg = tid % kTPR;
+    constexpr int OC = D / kTPR;  // output columns per thread
     for (int e = tid; e < kBM * D; e += kAttnSimtThreads) {
         const int rr = e / D, c = e % D, i = i0 + rr;
         sm.q[rr][c] = i < Lk ? Elem<T>::load(Q, qbase + (size_t)i * qstride + c) : 0.0f;
@@ -69,34 +74,34 @@ k_attn_simt(const T *__restrict__ Q, const T *__restrict__ K, const T *__restric
             sm.v[rr][c] = ok ? Elem<T>::load(V, kbase + (size_t)j * kstride + c) : 0.0f;
         }
         __syncthreads();
-        float s[16];
+        float s[kSC];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) s[c] = 0.0f;
+        for (int c = 0; c < kSC; ++c) s[c] = 0.0f;
         for (int k = 0; k < D; ++k) {
             const float qv = sm.q[r][k];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) s[c] = fmaf(qv, sm.k[cg * 16 + c][k], s[c]);
+            for (int c = 0; c < kSC; ++c) s[c] = fmaf(qv, sm.k[cg * kSC + c][k], s[c]);
         }
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const int j = j0 + cg * 16 + c;
+        for (int c = 0; c < kSC; ++c) {
+            const int j = j0 + cg * kSC + c;
             s[c] = (j <= i && j < Lk) ? s[c] * sl2 : -INFINITY;
             mx = fmaxf(mx, s[c]);
         }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+#pragma unroll
+        for (int o = 1; o < kTPR; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         const float mnew = fmaxf(m, mx);
         const float corr = (m == -INFINITY) ? 0.0f : exp2f(m - mnew);
         float ps = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < kSC; ++c) {
             const float p = (s[c] == -INFINITY) ? 0.0f : exp2f(s[c] - mnew);
-            sm.p[r][cg * 16 + c] = p;
+            sm.p[r][cg * kSC + c] = p;
             ps += p;
         }
-        ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+#pragma unroll
+        for (int o = 1; o < kTPR; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
         l = l * corr + ps;
         m = mnew;
 #pragma unroll

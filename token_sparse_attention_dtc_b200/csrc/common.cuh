@@ -17,7 +17,9 @@ struct Control {
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
-constexpr int kScoreSplitTokens = 4096;  // tokens per scoring split (SIMT path)
+// Tokens per scoring split of the CUDA-core path: 4096, fewer for shorter rows so that a
+// row still spans several blocks.
+inline int score_simt_split(int L) { return L >= 32768 ? 4096 : (L >= 4096 ? 1024 : 256); }
 // Scratch of the wave-scheduled tensor-core scoring: float2 per-CTA (max, sum) pairs of
 // 4 wave slots x up to 160 CTAs x 64 query rows, then float per-warp layer-score totals
 // [B][up to 160 CTAs][16 warps].
@@ -154,13 +156,13 @@ struct WsLayout {
 WsLayout ws_layout(const tsa_dims &dm, int q);
 
 // Capacity, per KV group, of the workspace's scoring splits: the CUDA-core path uses
-// ceil(L / 4096) splits, the tensor-core path at most ceil(256 / (B*Hkv)) (and no more
-// than the number of 128-token tiles).
+// ceil(L / score_simt_split(L)) splits, the tensor-core path at most ceil(256 / (B*Hkv))
+// (and no more than the number of 128-token tiles).
 inline int score_split_cap(const tsa_dims &dm) {
     const int groups = dm.B * dm.Hkv;
     const int tc = ceil_div(256, groups) < ceil_div(dm.L, 128) ? ceil_div(256, groups)
                                                               : ceil_div(dm.L, 128);
-    const int simt = ceil_div(dm.L, kScoreSplitTokens);
+    const int simt = ceil_div(dm.L, score_simt_split(dm.L));
     return simt > tc ? simt : tc;
 }
 

@@ -220,7 +220,7 @@ static cudaError_t score_simt_impl(const tsa_dims &dm, const void *Q, const void
                                    float scale, float *s_h, const WsLayout &w, char *ws,
                                    cudaStream_t st) {
     const float sl2 = scale * 1.4426950408889634f;
-    const int split_len = kScoreSplitTokens;
+    const int split_len = score_simt_split(dm.L);
     const int nsplit = ceil_div(dm.L, split_len);
     const int G = dm.H / dm.Hkv;
     float2 *part = reinterpret_cast<float2 *>(ws + w.score_part);
@@ -229,8 +229,15 @@ static cudaError_t score_simt_impl(const tsa_dims &dm, const void *Q, const void
     k_score_stats_simt<T, D><<<grid, kSimtThreads, 0, st>>>(
         (const T *)Q, (const T *)K, dm.L, dm.H, dm.Hkv, qe, sl2, split_len, nsplit, part);
     k_score_combine<<<dm.B * dm.Hkv, 256, 0, st>>>(part, nsplit, G * qe, stat);
-    k_score_colsum_simt<T, D, kScoreSplitTokens / kSimtThreads><<<grid, kSimtThreads, 0, st>>>(
-        (const T *)Q, (const T *)K, dm.L, dm.H, dm.Hkv, qe, sl2, split_len, stat, s_h);
+#define TSA_COLSUM(TPT)                                                                    \
+    k_score_colsum_simt<T, D, TPT><<<grid, kSimtThreads, 0, st>>>(                          \
+        (const T *)Q, (const T *)K, dm.L, dm.H, dm.Hkv, qe, sl2, split_len, stat, s_h)
+    switch (split_len / kSimtThreads) {  // tokens per thread
+        case 16: TSA_COLSUM(16); break;
+        case 4: TSA_COLSUM(4); break;
+        default: TSA_COLSUM(1); break;
+    }
+#undef TSA_COLSUM
     note_launches(3);
     return cudaGetLastError();
 }
