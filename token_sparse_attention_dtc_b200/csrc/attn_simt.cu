@@ -1,15 +1,15 @@
 // Causal attention on CUDA cores for fp32 inputs (the fp32 path keeps full fp32
 // products; tensor-core tf32 would not meet a 1e-4 output tolerance).  bf16 inputs run on
 // the tensor cores (attn_tc.cu).  Flash-style
-// online softmax over 64-key tiles, one block per (32-row query tile, batch, head).
+// online softmax over 64-key tiles, one block per (16-row query tile, batch, head).
 //
 // Method: "Token Sparse Attention" papernotes.org notes, 整体框架 (dense attention on
 // the compressed L'×L' problem); bxzpzcl.cn post §1.1 (softmax(Q̂K̂ᵀ/√d)V̂).  The causal
 // mask j <= i in compressed order equals the mask on original positions because the
 // index lists are ascending.
 //
-// 32-row query tiles (8 threads per row, each 8 key columns of S and D/8 output columns),
-// so that short rows still spread over many blocks.
+// 16-row query tiles (16 threads per row, each 4 key columns of S and D/16 output
+// columns), so that short rows still spread over many blocks.
 #include <math.h>
 
 #include "common.cuh"
@@ -17,7 +17,7 @@
 namespace tsa {
 
 constexpr int kAttnSimtThreads = 256;
-constexpr int kBM = 32, kBN = 64;
+constexpr int kBM = 16, kBN = 64;
 constexpr int kTPR = kAttnSimtThreads / kBM;  // threads per query row
 constexpr int kSC = kBN / kTPR;               // key columns of S per thread
 
