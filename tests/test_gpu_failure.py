@@ -87,6 +87,28 @@ def test_scoring_wait_timeout_is_reported_and_context_recovers(wave):
         torch.testing.assert_close(s_l, s_l_ref, rtol=1e-5, atol=1e-30)
 
 
+def test_one_wave_scoring_wait_timeout_is_reported_and_context_recovers():
+    """The automatic one-wave schedule (K of at least 192 MiB: 98304 tokens of the Llama
+    shape) times out the same way.  Its grid barrier and counters reset themselves at the
+    end of every launch, the timed-out one included, so the next launches give the first
+    launch's scores bit for bit."""
+    x = make_inputs(1, 98304, 32, 8, 128, torch.bfloat16, seed=41)
+    Q, K = x["Q"].cuda(), x["K"].cuda()
+    del x
+    dm = tsa.dims(Q, K)
+    ws = tsa.workspace(dm, 16)
+    ref_h, ref_l = (t.clone() for t in tsa.tsa_score(Q, K, 16, ws=ws))
+    assert tsa.tsa_get_device_status(ws) == 0
+    with stalled():
+        tsa.tsa_score(Q, K, 16, ws=ws)
+        st = tsa.tsa_get_device_status(ws)
+    assert st == TIMEOUT
+    for _ in range(2):
+        s_h, s_l = tsa.tsa_score(Q, K, 16, ws=ws)
+        assert tsa.tsa_get_device_status(ws) == 0
+        assert torch.equal(s_h, ref_h) and torch.equal(s_l, ref_l)
+
+
 def test_out_of_range_scores_are_flagged():
     """The budget and selection flag scores outside their legal range (NaN, < 0, or a
     layer score above 1) instead of using them silently."""
