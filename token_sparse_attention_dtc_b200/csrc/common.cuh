@@ -155,14 +155,14 @@ struct WsLayout {
 
 WsLayout ws_layout(const tsa_dims &dm, int q);
 
-// Capacity, per KV group, of the workspace's scoring splits: the CUDA-core path uses
-// ceil(L / score_simt_split(L)) splits, the tensor-core path at most ceil(256 / (B*Hkv))
-// (and no more than the number of 128-token tiles).
+// Capacity, per KV group, of the workspace's scoring splits: the CUDA-core path (fp32)
+// uses ceil(L / score_simt_split(L)) splits, the tensor-core path at most
+// ceil(256 / (B*Hkv)) (and no more than the number of 128-token tiles).
 inline int score_split_cap(const tsa_dims &dm) {
     const int groups = dm.B * dm.Hkv;
     const int tc = ceil_div(256, groups) < ceil_div(dm.L, 128) ? ceil_div(256, groups)
                                                               : ceil_div(dm.L, 128);
-    const int simt = ceil_div(dm.L, score_simt_split(dm.L));
+    const int simt = dm.dtype == TSA_F32 ? ceil_div(dm.L, score_simt_split(dm.L)) : 0;
     return simt > tc ? simt : tc;
 }
 
