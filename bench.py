@@ -43,14 +43,20 @@ def _peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def _traffic(kernel: str, workload: str):
+def _traffic_key(w, L: int):
+    """The traffic.json key of a workload run at length L: its name at its own length, none
+    when --L changed the size (a capture of another length does not apply)."""
+    return w.name if L == w.L else None
+
+
+def _traffic(kernel: str, workload):
     """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kernel, {}).get(workload)
+    e = d.get(kernel, {}).get(workload) if workload else None
     if not e:
         return None
     import hashlib
@@ -412,7 +418,7 @@ def run_ours(args, w, L, rank, world, local_rank):
             "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": attn_tf / peaks["bf16_sus"],
             "peak_kind": "bf16 sustained (%s)" % peaks["src"],
             "frac_of_burst": attn_tf / peaks["bf16"],
-            "traffic": _traffic("k_attn_tc", w.name)}
+            "traffic": _traffic("k_attn_tc", _traffic_key(w, L))}
     # HBM kernels: algorithmic bytes per launch
     H, dd = w.H, w.d
     hbm = {
@@ -431,7 +437,7 @@ def run_ours(args, w, L, rank, world, local_rank):
     score_kern = score_kernel_name(args.score_schedule, w, L)
     for k, kern in (("score", score_kern), ("gather", "k_gather_qkv"),
                     ("scatter", "k_scatter_residual")):
-        t = _traffic(kern, w.name)
+        t = _traffic(kern, _traffic_key(w, L))
         hbm_roof[k]["traffic"] = t
         hbm_roof[k]["dram_gbs"] = t / (stage_ms[k] * 1e-3) / 1e9 if t else None
         hbm_roof[k]["dram_frac"] = (t / (stage_ms[k] * 1e-3) / 1e9 / peaks["hbm"]) if t else None
@@ -1043,7 +1049,8 @@ def run_score_only(args, w, L):
                    "l2": "L2 flushed (512 MB written, then read) before each launch"},
         "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": pk["hbm"],
                      "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm"],
-                     "traffic": _traffic(kern, w.name), "algorithmic_bytes": nbytes}}),
+                     "traffic": _traffic(kern, _traffic_key(w, L)),
+                     "algorithmic_bytes": nbytes}}),
           flush=True)
 
 

@@ -88,6 +88,16 @@ def test_traffic_lookup_is_void_once_the_source_changes(tmp_path, monkeypatch):
     assert bench._traffic("k_x", "w") is None
 
 
+def test_traffic_key_applies_only_at_the_captured_length():
+    """A capture keyed by a workload name stands for that workload's own length; a run with
+    --L at another length reports no traffic."""
+    from token_sparse_attention_dtc_b200.inputs import WORKLOADS
+    w = WORKLOADS["llama8b_128k"]
+    assert bench._traffic_key(w, w.L) == "llama8b_128k"
+    assert bench._traffic_key(w, 98304) is None
+    assert bench._traffic("k_attn_tc", None) is None
+
+
 def test_peaks_read_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     fb = bench._peaks()
